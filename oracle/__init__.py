@@ -1,0 +1,112 @@
+"""CPU oracle for MLA decode attention over a paged latent KV cache.
+
+TEST INFRASTRUCTURE ONLY. This package is loaded by the test suite, by the smoke
+check in ``__graft_entry__`` and by the CPU-baseline leg of ``bench.py``; the
+product (the CUDA library under ``mla_decode_attention_14_b200``) never imports it,
+and the two share no code. The arithmetic lives in ``mla_oracle.c`` (plain C,
+double precision, POSIX threads); this module only builds and calls it.
+
+Sources: "Deep analysis of the DeepSeek Infra open-source releases"
+(jingzhunhuoke.net/55333.html), section "DAY1 FlashMLA" (MLA glossary entry,
+feature (2) 64-token KV blocks, feature (4) Gemm1/Gemm2, feature (5) variable
+lengths), plus the library's task statement for the dimensions (576-d keys, first
+512 dims as values), the scale, causal masking and output shapes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mla_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+D_QK = 576
+D_V = 512
+BLK = 64
+
+
+def build(force: bool = False) -> str:
+    """Compile ``mla_oracle.c`` into ``liboracle.so`` next to it (gcc, -O2)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".tmp.%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-Wall", "-Wextra",
+             "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        lib.oracle_metadata.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+        lib.oracle_metadata.restype = ctypes.c_int
+        lib.oracle_decode.argtypes = [P, P, ctypes.c_int64, P, ctypes.c_int64, P,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                      ctypes.c_int, P, P, P, ctypes.c_int64, ctypes.c_int]
+        lib.oracle_decode.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def metadata(seqlens, num_parts: int, fixed_cost: int):
+    """Work partition of every (sequence, 64-token block) into ``num_parts`` parts.
+
+    Returns ``(tile_meta int32[num_parts, 8], num_splits_cum int32[batch + 1])``;
+    the layout is documented in ``mla_oracle.c``.
+    """
+    s = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    tm = np.zeros((num_parts, 8), dtype=np.int32)
+    ns = np.zeros(s.shape[0] + 1, dtype=np.int32)
+    rc = _load().oracle_metadata(_ptr(s), int(s.shape[0]), int(num_parts), int(fixed_cost),
+                                 _ptr(tm), _ptr(ns))
+    if rc != 0:
+        raise ValueError("oracle_metadata: bad arguments (rc=%d)" % rc)
+    return tm, ns
+
+
+def decode(q_bits, kv_bits, block_table, seqlens, scale: float, causal: bool,
+           tasks=None, nthreads: int | None = None):
+    """Exact (double) MLA decode attention.
+
+    ``q_bits``: uint16 bf16 bit patterns ``[b, s_q, h_q, 576]``;
+    ``kv_bits``: uint16 ``[num_blocks, 64, 1, 576]`` (or ``[num_blocks, 64, 576]``);
+    ``block_table``: int32 ``[b, max_blocks]``; ``seqlens``: int32 ``[b]``.
+    Returns ``(out float64[b, s_q, h_q, 512], lse float64[b, h_q, s_q])``. With
+    ``tasks`` (int32 ``[k, 3]`` of (b, t, h)) only those rows are computed and the
+    others are NaN.
+    """
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kv = np.ascontiguousarray(kv_bits, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    b, s_q, h_q, d = q.shape
+    assert d == D_QK and kv.shape[-1] == D_QK and kv.shape[1] == BLK
+    nblk = kv.shape[0]
+    out = np.full((b, s_q, h_q, D_V), np.nan, dtype=np.float64)
+    lse = np.full((b, h_q, s_q), np.nan, dtype=np.float64)
+    if tasks is not None:
+        tk = np.ascontiguousarray(tasks, dtype=np.int32).reshape(-1, 3)
+        tptr, nt = _ptr(tk), tk.shape[0]
+    else:
+        tk, tptr, nt = None, None, 0
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().oracle_decode(_ptr(q), _ptr(kv), nblk, _ptr(bt), bt.shape[1] if bt.ndim == 2 else 0,
+                               _ptr(sl), b, s_q, h_q, float(scale), int(bool(causal)),
+                               _ptr(out), _ptr(lse), tptr, nt, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_decode failed (rc=%d)" % rc)
+    return out, lse
