@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Benchmark of MLA decode attention on B200: effective TB/s (KV + Q bytes) and TFLOPS.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3] [--impl ours|reference]
+
+One step = the whole decode path for one batch: split-KV metadata, the split kernel and
+the combine kernel, on inputs already resident in HBM (the KV cache, > 126 MB, is larger
+than L2, so no flush is needed between steps). Rank 0 prints one JSON line.
+
+Multi-GPU: one process per GPU (torchrun); every rank decodes its own batch of the same
+shape (independent problems, no collective on the data path: weak scaling); the time is
+the max over ranks and the value counts the bytes of all ranks.
+
+``--impl reference`` times the CPU oracle (the plain C fp64 implementation under
+``oracle/``) on a bounded sample of the same workload; it is the deliberately slow
+reference arm, run on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_decode_attention_14_b200 import workloads as W  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+METRIC = "MLA decode effective TB/s and TFLOPS vs B200 roofline (bf16 paged KV)"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_split_v3_traffic.txt")
+
+
+def describe(wl: W.Workload) -> str:
+    n = wl.seqlens
+    return ("%s: batch %d, h_q %d, s_q %d%s, seqlens %d..%d (mean %.0f), 64-token blocks, d_qk 576, d_v 512, "
+            "bf16 N(0,1), scale 192^-0.5" % (wl.name, wl.batch, wl.h_q, wl.s_q, " causal" if wl.causal else "",
+                                             n.min(), n.max(), n.mean()))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_decode_attention_14_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per split-kernel launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    try:
+        kv = {}
+        with open(PROFILE_TRAFFIC) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_sources_sha256_16") != kernel_source_hash():
+            return None
+        return float(kv["dram_bytes_per_launch_full_size"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 50):
+        self.index, self.period = index, period_ms
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() in ("active", "1"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, wl, inp, counts):
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    # calibrate: one row of the longest sequence
+    b_long = int(np.argmax(wl.seqlens))
+    t0 = time.perf_counter()
+    oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
+                  tasks=np.array([[b_long, 0, 0]], np.int32), nthreads=1)
+    per_row = max(time.perf_counter() - t0, 1e-4) * float(wl.seqlens.mean()) / float(wl.seqlens.max())
+    budget = min(10.0, 150.0 / max(1, args.steps + args.warmup))      # seconds of wall time per step
+    nrows = int(max(1, min(wl.h_q * wl.s_q, budget * cores / per_row)))
+    seq = int(rng.integers(0, wl.batch))
+    heads = np.arange(nrows) % wl.h_q
+    tasks = np.array([[seq, (i // wl.h_q) % wl.s_q, h] for i, h in enumerate(heads)], np.int32)
+    n = int(wl.seqlens[seq])
+    # algorithmic bytes of this sample: the sequence's KV once, plus its sampled query rows
+    sample_bytes = n * 1152 + nrows * 1152
+    for _ in range(args.warmup):
+        oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
+                      tasks=tasks, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
+                      tasks=tasks, nthreads=cores)
+    dt = (time.perf_counter() - t0) / args.steps
+    tbs = sample_bytes / dt / 1e12
+    sample = "%d of %d query rows of sequence %d (%d tokens), all its keys, per step" % (nrows, wl.rows, seq, n)
+    line = {"metric": METRIC, "value": tbs, "unit": "TB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": describe(wl), "sample": sample},
+            "cpu_baseline": {"value": tbs, "unit": "TB/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": tbs, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+def cpu_baseline(wl, inp, target_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the workload (rank 0, N = 1)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    seq = int(np.argsort(wl.seqlens)[len(wl.seqlens) // 2])   # a median-length sequence
+    n = int(wl.seqlens[seq])
+    t0 = time.perf_counter()
+    oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
+                  tasks=np.array([[seq, 0, 0]], np.int32), nthreads=1)
+    per_row = max(time.perf_counter() - t0, 1e-4)
+    nrows = int(max(cores, min(wl.rows, target_s * cores / per_row)))
+    tasks = np.array([[seq, (i // wl.h_q) % wl.s_q, i % wl.h_q] for i in range(nrows)], np.int32)
+    t0 = time.perf_counter()
+    oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
+                  tasks=tasks, nthreads=cores)
+    dt = time.perf_counter() - t0
+    # the metric's unit: algorithmic bytes (the sequence's KV once + sampled q rows) per second
+    val = (n * 1152 + nrows * 1152) / dt / 1e12
+    return {"value": val, "unit": "TB/s", "cores": cores, "kind": "oracle",
+            "sample": "%d of %d query rows of one %d-token sequence (all its keys), %.1f s" % (nrows, wl.rows, n, dt),
+            "seconds": dt}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="v3", choices=W.NAMES)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    wl = W.workload(args.workload)
+    counts = W.algorithmic_counts(wl)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inp = W.make_inputs(wl, seed=0, tail="normal")
+        run_reference(args, wl, inp, counts)
+        return
+
+    import torch
+    import mla_decode_attention_14_b200 as mla
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    inp = W.make_inputs(wl, seed=0, tail="normal")
+    dev = torch.device("cuda", local)
+    q = torch.from_numpy(inp["q"]).view(torch.bfloat16).to(dev)
+    kv = torch.from_numpy(inp["kv"]).view(torch.bfloat16).to(dev)
+    bt = torch.from_numpy(inp["block_table"]).to(dev)
+    sl = torch.from_numpy(inp["seqlens"]).to(dev)
+    num_parts = mla.default_num_parts(wl.h_q, wl.s_q, dev)
+    fixed_cost = mla.default_fixed_cost(wl.h_q, wl.s_q)
+    ws = torch.empty((mla.workspace_bytes(wl.batch, wl.s_q, wl.h_q, num_parts),), dtype=torch.uint8, device=dev)
+    out = torch.empty((wl.batch, wl.s_q, wl.h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.batch, wl.h_q, wl.s_q), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        meta = mla.get_metadata(sl, wl.h_q, wl.s_q, num_parts=num_parts, fixed_cost=fixed_cost)
+        if ev is not None:
+            ev[0].record(stream)
+        mla.decode(q, kv, bt, sl, wl.scale, wl.causal, meta, out=out, lse=lse, workspace=ws, phase="split")
+        if ev is not None:
+            ev[1].record(stream)
+        mla.decode(q, kv, bt, sl, wl.scale, wl.causal, meta, out=out, lse=lse, workspace=ws, phase="combine")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = mla.check_status()
+    if st != 0:
+        raise SystemExit("device error status %d after warm-up" % st)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = mla.launch_count()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    launches = mla.launch_count() - launches0
+    if dist is not None:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    split_ms = [a.elapsed_time(b) for a, b in evs]
+    st = mla.check_status()
+    if st != 0:
+        raise SystemExit("device error status %d in the timed region" % st)
+
+    if dist is not None:
+        t = torch.tensor([total_ms, statistics.mean(split_ms)], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, split_avg_ms = float(t[0]), float(t[1])
+    else:
+        split_avg_ms = statistics.mean(split_ms)
+    ms_per_step = total_ms / args.steps
+    bytes_all = counts["bytes"] * world
+    value = bytes_all / (ms_per_step * 1e-3) / 1e12
+    tflops = counts["flops"] * world / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the host entry point: pinned host inputs in, host outputs out
+    e2e = None
+    if args.e2e_steps > 0:
+        hd = mla.HostDecoder(wl.batch, wl.s_q, wl.h_q, kv.shape[0], bt.shape[1], device=dev,
+                             num_parts=num_parts, fixed_cost=fixed_cost)
+        qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
+        kvh = torch.from_numpy(inp["kv"]).view(torch.bfloat16).pin_memory()
+        bth = torch.from_numpy(inp["block_table"]).pin_memory()
+        slh = torch.from_numpy(inp["seqlens"]).pin_memory()
+        oh = torch.empty(tuple(out.shape), dtype=torch.bfloat16).pin_memory()
+        lh = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+        for _ in range(2):
+            hd(qh, kvh, bth, slh, wl.scale, wl.causal, oh, lh)
+        if dist is not None:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            hd(qh, kvh, bth, slh, wl.scale, wl.causal, oh, lh)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        h2d = sum(x.numel() * x.element_size() for x in (qh, kvh, bth, slh))
+        d2h = oh.numel() * 2 + lh.numel() * 4
+        e2e = {"value": bytes_all / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0:
+        hbm, tfl_burst, tfl_sust, src = measured_peaks()
+        ai = counts["flops"] / counts["bytes"]
+        ridge = tfl_burst * 1e12 / (hbm * 1e9)
+        split_s = split_avg_ms * 1e-3
+        ach_gbs = counts["bytes"] / split_s / 1e9
+        ach_tf = counts["flops"] / split_s / 1e12
+        bound = "hbm" if ai < ridge else "tensor"
+        if bound == "hbm":
+            roof = {"bound": "hbm", "achieved": ach_gbs, "peak": hbm, "unit": "GB/s", "frac": ach_gbs / hbm}
+        else:
+            roof = {"bound": "tensor", "achieved": ach_tf, "peak": tfl_burst, "unit": "TFLOP/s",
+                    "frac": ach_tf / tfl_burst}
+        roof.update({"traffic": profiled_traffic(), "kernel": "mla decode split kernel",
+                     "peak_source": src + " (MEASURED_PEAKS.json)" if src == "measured" else "fallback",
+                     "algorithmic_bytes_per_launch": counts["bytes"], "algorithmic_flops_per_launch": counts["flops"],
+                     "launch_ms": split_avg_ms, "hbm_frac": ach_gbs / hbm, "tensor_frac": ach_tf / tfl_burst,
+                     "tensor_frac_sustained": ach_tf / tfl_sust})
+        line = {"metric": METRIC, "value": value, "unit": "TB/s", "tflops": tflops, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": describe(wl), "batch": wl.batch, "h_q": wl.h_q, "s_q": wl.s_q,
+                           "causal": wl.causal, "num_parts": num_parts, "fixed_cost": fixed_cost,
+                           "l2": "inputs larger than L2 (KV cache %.0f MB > 126 MB); no flush" % (counts["kv_bytes"] / 1e6),
+                           "parallelism": "independent batch per GPU" if world > 1 else "1 GPU"},
+                "roofline": roof, "clocks": clk.summary(), "e2e": e2e, "gpu_launches": launches}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, inp)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,195 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) MLA decode-attention library.
+ *
+ * What is computed. Multi-head Latent Attention (MLA) decoding over a paged latent
+ * KV cache. MLA is the attention of DeepSeek-V2 that replaces GQA, and FlashMLA is a
+ * FlashAttention-style CUDA kernel for it ("Deep analysis of the DeepSeek Infra
+ * open-source releases", jingzhunhuoke.net/55333.html, section "DAY1 FlashMLA",
+ * glossary). Every query head attends over ONE shared 576-d latent vector per token
+ * (512 compressed dims + 64 rotary dims). The key is the whole 576-d vector, the value
+ * is its first 512 dims. The cache is stored in blocks of 64 tokens (same section,
+ * feature (2)) addressed through a per-sequence block table. For batch b, query token
+ * t, head h (row r = t*h_q + h):
+ *     n  = seqlens[b]
+ *     V  = causal ? clamp(n - s_q + t + 1, 0, n) : n        (visible keys)
+ *     k_j = kv_cache[block_table[b*bt_stride + j/64]][j%64][0][0:576],  j < V
+ *     s_j = scale * <q[b][t][h][:], k_j>
+ *     lse[b][h][t]       = log(sum_j exp(s_j))               (natural log)
+ *     out[b][t][h][0:512] = sum_j exp(s_j - lse) * k_j[0:512]
+ *     V == 0  ->  out = 0, lse = -inf
+ * The pages do not write this formula out; it is the standard scaled-softmax reading.
+ * The query tokens of one sequence are its last s_q tokens under causal masking.
+ *
+ * How. Two steps on the caller's stream:
+ *   1. mla_get_metadata: a length-aware split of all (sequence, 64-token block) work
+ *      into `num_parts` contiguous parts (same section, feature (5): inputs of very
+ *      different lengths are load-balanced). A sequence that spans k > 1 parts is
+ *      computed as k pieces.
+ *   2. mla_decode: a persistent kernel walks each part (one 2-CTA cluster per part and
+ *      group of 128 query rows): TMA gathers of block-table-addressed KV tiles into a
+ *      shared-memory ring, QK^T ("Gemm1") and PV ("Gemm2") as tcgen05 MMAs with TMEM
+ *      accumulators (same section, feature (4)), an fp32 online softmax; pieces of
+ *      split sequences leave fp32 partial outputs + lse in the workspace, and a
+ *      combine kernel merges them by log-sum-exp.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers unless the name says host. All device buffers are
+ *     owned by the caller; the library allocates no device memory. It keeps only a
+ *     small host-side cache of TMA descriptors keyed by (kv_cache, num_blocks).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous unless stated; nothing is synchronised implicitly.
+ *   - Inputs are never written. Arguments are validated on the host BEFORE any launch;
+ *     an invalid call returns a non-zero mla_status and launches nothing.
+ *   - Kernels never trap. A block-table entry outside [0, num_blocks) or a pipeline
+ *     wait that exceeds its iteration bound sets a per-device error word; the affected
+ *     outputs are then unspecified. mla_check_status() reports and clears it.
+ *   - Thread safety: calls on different streams may run concurrently; the TMA
+ *     descriptor cache is guarded by a mutex.
+ */
+#ifndef MLA_DECODE_B200_MLA_H_
+#define MLA_DECODE_B200_MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_D_QK 576          /* key width: 512 latent + 64 rotary dims        */
+#define MLA_D_V 512           /* value width: the first 512 dims of the key    */
+#define MLA_BLOCK_TOKENS 64   /* tokens per cache block                        */
+#define MLA_TILE_META_INTS 8  /* int32 per part in tile_meta                   */
+#define MLA_MAX_ROWS 1024     /* max s_q * h_q per call                        */
+#define MLA_MAX_BATCH 65536   /* max batch per call                            */
+
+typedef enum mla_status {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, size out of range        */
+    MLA_ERR_UNSUPPORTED = 2, /* device is not sm_100 / shape not supported        */
+    MLA_ERR_WORKSPACE = 3,   /* workspace smaller than mla_workspace_bytes()      */
+    MLA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                 */
+    MLA_ERR_TIMEOUT = 5,     /* a device pipeline wait hit its bound (reported by mla_check_status) */
+    MLA_ERR_BOUNDS = 6       /* a block-table entry outside [0, num_blocks) was needed */
+} mla_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *mla_status_string(int status);
+
+/*
+ * Default number of parts for the decode kernel on `device`: one part per 2-SM cluster
+ * per group of 128 query rows, i.e. floor(SMs / 2) / ceil(s_q*h_q / 128), at least 1.
+ * Host only (queries the SM count). Returns MLA_OK and writes *num_parts.
+ */
+int mla_default_num_parts(int device, int h_q, int s_q, int *num_parts);
+
+/* Default per-piece start-up cost, in 64-token-block units, used by the partition. */
+int mla_default_fixed_cost(int h_q, int s_q);
+
+/*
+ * Bytes of device workspace mla_decode needs: fp32 partial outputs and lse for at most
+ * batch + num_parts - 1 pieces of s_q*h_q rows each:
+ *     (batch + num_parts) * s_q * h_q * (512 + 1) * 4, rounded up to 256.
+ * Returns 0 for invalid sizes. Host only.
+ */
+size_t mla_workspace_bytes(int batch, int s_q, int h_q, int num_parts);
+
+/*
+ * Split-KV metadata ("tile-scheduler metadata").
+ *   seqlens     int32[batch]                  device, read only (negative = 0)
+ *   tile_meta   int32[num_parts * 8]          device, written: per part
+ *               {begin_seq, begin_blk, end_seq (inclusive), end_blk (exclusive),
+ *                index of the part's first piece within its sequence, 0, 0, 0};
+ *               an empty part is {0, 0, -1, 0, 0, 0, 0, 0}
+ *   num_splits  int32[batch + 1]              device, written: num_splits[0] = 0,
+ *               num_splits[i+1] - num_splits[i] = pieces of sequence i (0 if n_i <= 0)
+ *   fixed_cost  start-up cost of a sequence in block units (>= 0)
+ * Rule: sequence i with w_i = ceil(n_i/64) > 0 blocks occupies fixed_cost + w_i units on a
+ * line of work units (start-up first, then its blocks, sequences in order); with U units
+ * in all, T = max(1, ceil(U/num_parts)) and the block at unit u belongs to part u / T.
+ * One single-CTA launch; h_q and s_q are validated but do not change the result.
+ */
+int mla_get_metadata(const int32_t *seqlens, int batch, int h_q, int s_q, int num_parts,
+                     int fixed_cost, int32_t *tile_meta, int32_t *num_splits, void *stream);
+
+/*
+ * Decode attention (split kernel + combine kernel on `stream`).
+ *   q            bf16[batch, s_q, h_q, 576]      contiguous, 16-byte aligned
+ *   kv_cache     bf16[num_blocks, 64, 1, 576]    contiguous, 16-byte aligned
+ *   block_table  int32[batch, bt_stride]          entry j of row b = physical block of
+ *                tokens [64j, 64j+64) of sequence b; only the first ceil(n_b/64) entries
+ *                are read; others may hold anything (e.g. -1)
+ *   seqlens      int32[batch]                     tokens in each sequence (<= 64*bt_stride)
+ *   tile_meta, num_splits, num_parts, as produced by mla_get_metadata for these seqlens
+ *   scale        multiplies q.k before the softmax (finite)
+ *   causal       0/1, masking between the s_q query tokens (see top of file)
+ *   out          bf16[batch, s_q, h_q, 512]       written (round to nearest even)
+ *   lse          fp32[batch, h_q, s_q]            written (natural log; -inf if no key)
+ *   workspace    >= mla_workspace_bytes(batch, s_q, h_q, num_parts) bytes, 256-aligned;
+ *                contents on entry are ignored
+ * Requires an sm_100 device (B200). 1 <= s_q*h_q <= MLA_MAX_ROWS.
+ */
+int mla_decode(const void *q, const void *kv_cache, int64_t num_blocks,
+               const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+               const int32_t *tile_meta, const int32_t *num_splits, int num_parts, int batch,
+               int s_q, int h_q, float scale, int causal, void *out, float *lse,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/* The two launches of mla_decode, separately (same arguments and rules). The split
+ * kernel writes `out`/`lse` of every sequence held by one piece and the workspace
+ * partials of the others; the combine kernel then finishes the split sequences and
+ * the sequences with no tokens. Both must run, in this order, on the same stream. */
+int mla_decode_split(const void *q, const void *kv_cache, int64_t num_blocks,
+                     const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                     const int32_t *tile_meta, const int32_t *num_splits, int num_parts,
+                     int batch, int s_q, int h_q, float scale, int causal, void *out,
+                     float *lse, void *workspace, size_t workspace_bytes, void *stream);
+int mla_decode_combine(const int32_t *num_splits, int num_parts, int batch, int s_q, int h_q,
+                       void *out, float *lse, const void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/*
+ * End-to-end call on HOST buffers: copies the inputs host->device, runs metadata +
+ * decode, copies out/lse device->host, and synchronises `stream` before returning.
+ * Host buffers should be pinned for the copies to be asynchronous. `dev` holds the
+ * caller-allocated device buffers, each at least as large as the host one
+ * (workspace: mla_workspace_bytes). Uses num_parts = dev->num_parts and
+ * fixed_cost = dev->fixed_cost.
+ */
+typedef struct mla_device_buffers {
+    void *q;             /* bf16[batch, s_q, h_q, 576]    */
+    void *kv_cache;      /* bf16[num_blocks, 64, 1, 576]  */
+    int32_t *block_table;/* int32[batch, bt_stride]       */
+    int32_t *seqlens;    /* int32[batch]                  */
+    int32_t *tile_meta;  /* int32[num_parts * 8]          */
+    int32_t *num_splits; /* int32[batch + 1]              */
+    void *out;           /* bf16[batch, s_q, h_q, 512]    */
+    float *lse;          /* fp32[batch, h_q, s_q]         */
+    void *workspace;
+    size_t workspace_bytes;
+    int num_parts;
+    int fixed_cost;
+} mla_device_buffers;
+
+int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_blocks,
+                    const int32_t *block_table_host, int64_t bt_stride,
+                    const int32_t *seqlens_host, int batch, int s_q, int h_q, float scale,
+                    int causal, void *out_host, float *lse_host,
+                    const mla_device_buffers *dev, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's error word.
+ * Returns MLA_OK, MLA_ERR_BOUNDS, MLA_ERR_TIMEOUT, or MLA_ERR_CUDA if a CUDA call
+ * (including an earlier asynchronous launch) failed.
+ */
+int mla_check_status(void *stream);
+
+/* Number of kernel launches made by this process through the library so far (host
+ * counter; used to report how many of the library's kernels a benchmark ran). */
+int64_t mla_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_B200_MLA_H_ */

@@ -1,1 +1,268 @@
-"""B200-native MLA decode attention over a paged latent KV cache (placeholder; binding follows)."""
+"""B200-native (sm_100a) MLA decode attention over a paged latent KV cache.
+
+Thin Python binding of the C ABI in ``include/mla.h`` (``libmla_b200.so``, built in-tree by
+``python -m mla_decode_attention_14_b200.build``). It only marshals arguments: every step of
+the computation runs in the library's CUDA kernels. PyTorch provides device memory and
+streams. There is no CPU or framework fallback: if the library is missing or the device is
+not an sm_100 GPU, the calls raise.
+
+    meta = get_metadata(seqlens, h_q, s_q)              # split-KV schedule (device int32)
+    out, lse = decode(q, kv_cache, block_table, seqlens, scale, causal, meta)
+
+Shapes: q bf16 [b, s_q, h_q, 576]; kv_cache bf16 [num_blocks, 64, 1, 576] (64-token blocks,
+"Deep analysis of the DeepSeek Infra open-source releases", DAY1 FlashMLA, feature (2));
+block_table int32 [b, max_blocks]; seqlens int32 [b]; out bf16 [b, s_q, h_q, 512];
+lse fp32 [b, h_q, s_q].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+D_QK = 576
+D_V = 512
+BLOCK = 64
+META_INTS = 8
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+_lib = None
+
+MLA_OK = 0
+STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_WORKSPACE",
+                4: "MLA_ERR_CUDA", 5: "MLA_ERR_TIMEOUT", 6: "MLA_ERR_BOUNDS"}
+
+# exported C symbols, in the order include/mla.h declares them
+EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
+           "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_host",
+           "mla_check_status", "mla_launch_count")
+
+
+class MLAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = lib().mla_status_string(status).decode() if _lib is not None else STATUS_NAMES.get(status, "?")
+        super().__init__("%s failed: %s (status %d)" % (fn, msg, status))
+
+
+class _DeviceBuffers(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("kv_cache", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("seqlens", ctypes.c_void_p), ("tile_meta", ctypes.c_void_p), ("num_splits", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t), ("num_parts", ctypes.c_int), ("fixed_cost", ctypes.c_int)]
+
+
+def lib():
+    """Load ``libmla_b200.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libmla_b200.so not found at %s; build it with "
+                               "`python -m mla_decode_attention_14_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+        L.mla_status_string.argtypes = [I]
+        L.mla_status_string.restype = ctypes.c_char_p
+        L.mla_default_num_parts.argtypes = [I, I, I, ctypes.POINTER(I)]
+        L.mla_default_num_parts.restype = I
+        L.mla_default_fixed_cost.argtypes = [I, I]
+        L.mla_default_fixed_cost.restype = I
+        L.mla_workspace_bytes.argtypes = [I, I, I, I]
+        L.mla_workspace_bytes.restype = SZ
+        L.mla_get_metadata.argtypes = [P, I, I, I, I, I, P, P, P]
+        L.mla_get_metadata.restype = I
+        dec = [P, P, I64, P, I64, P, P, P, I, I, I, I, F, I, P, P, P, SZ, P]
+        for name in ("mla_decode", "mla_decode_split"):
+            getattr(L, name).argtypes = dec
+            getattr(L, name).restype = I
+        L.mla_decode_combine.argtypes = [P, I, I, I, I, P, P, P, SZ, P]
+        L.mla_decode_combine.restype = I
+        L.mla_decode_host.argtypes = [P, P, I64, P, I64, P, I, I, I, F, I, P, P,
+                                      ctypes.POINTER(_DeviceBuffers), P]
+        L.mla_decode_host.restype = I
+        L.mla_check_status.argtypes = [P]
+        L.mla_check_status.restype = I
+        L.mla_launch_count.argtypes = []
+        L.mla_launch_count.restype = I64
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != MLA_OK:
+        raise MLAError(fn, rc)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim=None, cuda=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if cuda and not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got shape %s" % (name, ndim, tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+@dataclass
+class Metadata:
+    """Split-KV schedule produced by :func:`get_metadata` (device tensors)."""
+    tile_meta: torch.Tensor   # int32 [num_parts, 8]
+    num_splits: torch.Tensor  # int32 [batch + 1], cumulative piece counts
+    num_parts: int
+    fixed_cost: int
+    h_q: int
+    s_q: int
+
+
+def default_num_parts(h_q: int, s_q: int, device=None) -> int:
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index or 0
+    n = ctypes.c_int(0)
+    _check("mla_default_num_parts", lib().mla_default_num_parts(dev, h_q, s_q, ctypes.byref(n)))
+    return n.value
+
+
+def default_fixed_cost(h_q: int, s_q: int) -> int:
+    return lib().mla_default_fixed_cost(h_q, s_q)
+
+
+def workspace_bytes(batch: int, s_q: int, h_q: int, num_parts: int) -> int:
+    return lib().mla_workspace_bytes(batch, s_q, h_q, num_parts)
+
+
+def get_metadata(seqlens: torch.Tensor, h_q: int, s_q: int, num_parts: int | None = None,
+                 fixed_cost: int | None = None, stream=None) -> Metadata:
+    """Tile-scheduler metadata and per-sequence split counts for ``seqlens`` (int32 [b], CUDA)."""
+    _need(seqlens, "seqlens", torch.int32, 1)
+    b = seqlens.shape[0]
+    if num_parts is None:
+        num_parts = default_num_parts(h_q, s_q, seqlens.device)
+    if fixed_cost is None:
+        fixed_cost = default_fixed_cost(h_q, s_q)
+    tm = torch.empty((num_parts, META_INTS), dtype=torch.int32, device=seqlens.device)
+    ns = torch.empty((b + 1,), dtype=torch.int32, device=seqlens.device)
+    with torch.cuda.device(seqlens.device):
+        _check("mla_get_metadata", lib().mla_get_metadata(seqlens.data_ptr(), b, h_q, s_q, num_parts, fixed_cost,
+                                                          tm.data_ptr(), ns.data_ptr(), _stream(stream)))
+    return Metadata(tm, ns, num_parts, fixed_cost, h_q, s_q)
+
+
+def _decode_args(q, kv_cache, block_table, seqlens, meta):
+    _need(q, "q", torch.bfloat16, 4)
+    _need(kv_cache, "kv_cache", torch.bfloat16)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    b, s_q, h_q, d = q.shape
+    if d != D_QK:
+        raise ValueError("q last dim must be %d" % D_QK)
+    if kv_cache.dim() == 4:
+        if kv_cache.shape[1:] != (BLOCK, 1, D_QK):
+            raise ValueError("kv_cache must be [num_blocks, 64, 1, 576], got %s" % (tuple(kv_cache.shape),))
+    elif kv_cache.dim() != 3 or kv_cache.shape[1:] != (BLOCK, D_QK):
+        raise ValueError("kv_cache must be [num_blocks, 64, 1, 576], got %s" % (tuple(kv_cache.shape),))
+    if block_table.shape[0] != b or seqlens.shape[0] != b:
+        raise ValueError("batch mismatch between q, block_table and seqlens")
+    if meta.h_q != h_q or meta.s_q != s_q or meta.num_splits.shape[0] != b + 1:
+        raise ValueError("metadata was computed for another shape")
+    return b, s_q, h_q
+
+
+def decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+           scale: float, causal: bool, meta: Metadata, out: torch.Tensor | None = None,
+           lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None,
+           phase: str = "both"):
+    """MLA decode attention; returns ``(out bf16 [b, s_q, h_q, 512], lse fp32 [b, h_q, s_q])``.
+
+    ``phase`` = "split" or "combine" runs one of the two kernels only (for timing each).
+    """
+    b, s_q, h_q = _decode_args(q, kv_cache, block_table, seqlens, meta)
+    dev = q.device
+    if out is None:
+        out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    ws_bytes = workspace_bytes(b, s_q, h_q, meta.num_parts)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    if workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError("workspace too small: need %d bytes" % ws_bytes)
+    st = _stream(stream)
+    L = lib()
+    with torch.cuda.device(dev):
+        if phase in ("both", "split"):
+            fn = L.mla_decode if phase == "both" else L.mla_decode_split
+            _check("mla_decode", fn(q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(),
+                                    block_table.shape[1], seqlens.data_ptr(), meta.tile_meta.data_ptr(),
+                                    meta.num_splits.data_ptr(), meta.num_parts, b, s_q, h_q, float(scale),
+                                    int(bool(causal)), out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                    ws_bytes, st))
+        elif phase == "combine":
+            _check("mla_decode_combine", L.mla_decode_combine(meta.num_splits.data_ptr(), meta.num_parts, b, s_q,
+                                                              h_q, out.data_ptr(), lse.data_ptr(),
+                                                              workspace.data_ptr(), ws_bytes, st))
+        else:
+            raise ValueError(phase)
+    return out, lse
+
+
+class HostDecoder:
+    """End-to-end decode on host buffers through ``mla_decode_host`` (copies in, runs, copies out).
+
+    Device buffers are allocated once (by torch) for the largest shapes given.
+    """
+
+    def __init__(self, batch, s_q, h_q, num_blocks, bt_stride, device="cuda", num_parts=None, fixed_cost=None):
+        dev = torch.device(device)
+        self.device = dev
+        self.num_parts = num_parts or default_num_parts(h_q, s_q, dev)
+        self.fixed_cost = default_fixed_cost(h_q, s_q) if fixed_cost is None else fixed_cost
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)  # noqa: E731
+        self.q = e((batch, s_q, h_q, D_QK), torch.bfloat16)
+        self.kv = e((num_blocks, BLOCK, 1, D_QK), torch.bfloat16)
+        self.bt = e((batch, bt_stride), torch.int32)
+        self.sl = e((batch,), torch.int32)
+        self.tm = e((self.num_parts, META_INTS), torch.int32)
+        self.ns = e((batch + 1,), torch.int32)
+        self.out = e((batch, s_q, h_q, D_V), torch.bfloat16)
+        self.lse = e((batch, h_q, s_q), torch.float32)
+        self.ws_bytes = workspace_bytes(batch, s_q, h_q, self.num_parts)
+        self.ws = e((self.ws_bytes,), torch.uint8)
+        self.buf = _DeviceBuffers(self.q.data_ptr(), self.kv.data_ptr(), self.bt.data_ptr(), self.sl.data_ptr(),
+                                  self.tm.data_ptr(), self.ns.data_ptr(), self.out.data_ptr(), self.lse.data_ptr(),
+                                  self.ws.data_ptr(), self.ws_bytes, self.num_parts, self.fixed_cost)
+
+    def __call__(self, q, kv_cache, block_table, seqlens, scale, causal, out, lse, stream=None):
+        """Host tensors in (pinned CPU torch tensors), host tensors out; synchronous."""
+        for t, n in ((q, "q"), (kv_cache, "kv_cache"), (block_table, "block_table"), (seqlens, "seqlens"),
+                     (out, "out"), (lse, "lse")):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("%s must be a contiguous host tensor" % n)
+        b, s_q, h_q, _ = q.shape
+        with torch.cuda.device(self.device):
+            _check("mla_decode_host", lib().mla_decode_host(
+                q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(), block_table.shape[1],
+                seqlens.data_ptr(), b, s_q, h_q, float(scale), int(bool(causal)), out.data_ptr(), lse.data_ptr(),
+                ctypes.byref(self.buf), _stream(stream)))
+        return out, lse
+
+
+def check_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status (0 = OK)."""
+    return lib().mla_check_status(_stream(stream))
+
+
+def launch_count() -> int:
+    """Kernels launched through the library by this process so far."""
+    return int(lib().mla_launch_count())

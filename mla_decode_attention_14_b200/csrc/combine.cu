@@ -1,0 +1,96 @@
+// combine.cu -- merges the partial results of sequences computed as several pieces.
+//
+// A piece s of a sequence leaves, per query row, o_s = (sum_j e^{s_j} v_j) / (sum_j e^{s_j})
+// over its keys and lse_s = log(sum_j e^{s_j}). The whole-sequence result is
+//   lse = log(sum_s e^{lse_s}),   out = sum_s e^{lse_s - lse} o_s
+// (the split-KV reading of "Deep analysis of the DeepSeek Infra open-source releases",
+// DAY1 FlashMLA, feature (5); the merge is exact up to rounding). Pieces with no visible
+// key carry lse_s = -inf and weight 0; if every piece of a row is empty the row gets
+// out = 0, lse = -inf. Sequences with no tokens at all (no piece) are written here too.
+//
+// One warp per (sequence, row); each lane owns 16 of the 512 output dims (four float4),
+// so every partial row is read as one coalesced 2 KB segment.
+#include "common.cuh"
+
+namespace mla {
+
+constexpr int kCombineWarps = 8;
+
+__global__ void __launch_bounds__(kCombineWarps * 32)
+combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts, int s_q, int h_q,
+               __nv_bfloat16 *__restrict__ out, float *__restrict__ lse,
+               const float *__restrict__ o_part, const float *__restrict__ lse_part) {
+    const int rows = s_q * h_q;
+    const int b = blockIdx.x;
+    const int r = blockIdx.y * kCombineWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (b >= batch || r >= rows) return;
+    const int s0 = num_splits[b], s1 = num_splits[b + 1];
+    const int ns = s1 - s0;
+    if (ns == 1) return;  // written directly by the split kernel
+    if (ns < 0 || s0 < 0 || s1 > batch + num_parts) {  // malformed metadata
+        if (lane == 0) raise_error(kErrBounds);
+        return;
+    }
+    const int t = r / h_q, h = r % h_q;
+    __nv_bfloat16 *orow = out + ((size_t)b * rows + r) * kDv + lane * 16;
+    float *lrow = lse + ((size_t)b * h_q + h) * s_q + t;
+
+    float m = -INFINITY;
+    for (int s = lane; s < ns; s += 32) m = fmaxf(m, lse_part[(size_t)(s0 + s) * rows + r]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+
+    if (ns == 0 || m == -INFINITY) {
+        uint4 z = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4 *>(orow)[0] = z;
+        reinterpret_cast<uint4 *>(orow)[1] = z;
+        if (lane == 0) *lrow = -INFINITY;
+        return;
+    }
+    float sum = 0.f;
+    for (int s = lane; s < ns; s += 32) sum += expf(lse_part[(size_t)(s0 + s) * rows + r] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float L = m + logf(sum);
+
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    for (int s = 0; s < ns; ++s) {
+        const size_t slot = (size_t)(s0 + s) * rows + r;
+        const float wgt = expf(lse_part[slot] - L);
+        if (wgt == 0.f) continue;  // empty piece (its o is 0) or negligible weight
+        const float4 *src = reinterpret_cast<const float4 *>(o_part + slot * kDv + lane * 16);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float4 v = src[k];
+            acc[4 * k + 0] += wgt * v.x;
+            acc[4 * k + 1] += wgt * v.y;
+            acc[4 * k + 2] += wgt * v.z;
+            acc[4 * k + 3] += wgt * v.w;
+        }
+    }
+    uint4 packed[2];
+    uint32_t *pw = reinterpret_cast<uint32_t *>(packed);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        __nv_bfloat162 two = __floats2bfloat162_rn(acc[2 * k], acc[2 * k + 1]);
+        pw[k] = *reinterpret_cast<uint32_t *>(&two);
+    }
+    reinterpret_cast<uint4 *>(orow)[0] = packed[0];
+    reinterpret_cast<uint4 *>(orow)[1] = packed[1];
+    if (lane == 0) *lrow = L;
+}
+
+cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q,
+                           __nv_bfloat16 *out, float *lse, const float *o_part,
+                           const float *lse_part, cudaStream_t stream) {
+    const int rows = s_q * h_q;
+    dim3 grid(batch, (rows + kCombineWarps - 1) / kCombineWarps);
+    combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(num_splits, batch, num_parts, s_q, h_q, out, lse,
+                                                           o_part, lse_part);
+    return cudaGetLastError();
+}
+
+}  // namespace mla

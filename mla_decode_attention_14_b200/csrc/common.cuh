@@ -1,0 +1,54 @@
+// common.cuh -- device-side helpers shared by the library's kernels (not by any test code).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mla {
+
+constexpr int kDqk = 576;        // key width: 512 latent + 64 rotary dims
+constexpr int kDv = 512;         // value width: first 512 dims of the key
+constexpr int kBlk = 64;         // tokens per cache block
+constexpr int kMetaInts = 8;     // int32 per part in tile_meta
+
+// Per-device error word (bit flags), read and cleared by mla_check_status().
+constexpr unsigned kErrBounds = 1u;   // a needed block-table entry was outside [0, num_blocks)
+constexpr unsigned kErrTimeout = 2u;  // a pipeline wait hit its iteration bound
+// Defined here: the library is one translation unit (csrc/mla_lib.cu).
+__device__ unsigned int g_error_word = 0;
+
+__device__ __forceinline__ void raise_error(unsigned bit) { atomicOr(&g_error_word, bit); }
+
+// Parameters shared by the split kernels (one struct, passed by value).
+struct DecodeParams {
+    const __nv_bfloat16 *q;        // [b, s_q, h_q, 576]
+    const __nv_bfloat16 *kv;       // [nblk, 64, 576]
+    const int32_t *block_table;    // [b, bt_stride]
+    const int32_t *seqlens;        // [b]
+    const int32_t *tile_meta;      // [num_parts, 8]
+    const int32_t *num_splits;     // [b + 1] (cumulative)
+    __nv_bfloat16 *out;            // [b, s_q, h_q, 512]
+    float *lse;                    // [b, h_q, s_q]
+    float *o_part;                 // [slots, rows, 512]
+    float *lse_part;               // [slots, rows]
+    int64_t num_blocks;
+    int64_t bt_stride;
+    int batch, s_q, h_q, rows, num_parts;
+    int causal;
+    float scale;                   // softmax scale
+    float scale_log2;              // scale * log2(e)
+};
+
+// Visible keys of query token t in a sequence of n tokens (causal: the s_q query
+// tokens are the sequence's last s_q tokens).
+__device__ __forceinline__ int visible_keys(int n, int s_q, int t, int causal) {
+    if (n < 0) n = 0;
+    if (!causal) return n;
+    int v = n - s_q + t + 1;
+    return v < 0 ? 0 : (v > n ? n : v);
+}
+
+__device__ __forceinline__ int num_blocks_of(int n) { return n > 0 ? (n + kBlk - 1) / kBlk : 0; }
+
+}  // namespace mla

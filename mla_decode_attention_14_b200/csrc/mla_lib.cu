@@ -1,0 +1,6 @@
+// mla_lib.cu -- single translation unit of the library (the device error word and all
+// kernels live in one module, so no separate device linking is needed).
+#include "api.cu"
+#include "metadata.cu"
+#include "combine.cu"
+#include "decode_simt.cu"

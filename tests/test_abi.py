@@ -1,0 +1,100 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol include/mla.h
+declares, and rejects invalid arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mla_decode_attention_14_b200 as mla
+from mla_decode_attention_14_b200 import build as mla_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    mla_build.build()
+    return mla.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(mla.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_library_links_no_cuda_driver_at_load_time():
+    # the runtime is static and driver entry points are resolved lazily, so the .so
+    # loads on a machine without a GPU driver
+    import subprocess
+    out = subprocess.run(["ldd", mla.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+
+
+def test_status_strings(L):
+    for code, name in mla.STATUS_NAMES.items():
+        assert L.mla_status_string(code).decode().startswith(name)
+    assert L.mla_status_string(99).decode() == "MLA: unknown status"
+
+
+def test_workspace_formula(L):
+    b, s_q, h_q, P = 128, 1, 128, 74
+    raw = (b + P) * s_q * h_q * (512 + 1) * 4
+    assert L.mla_workspace_bytes(b, s_q, h_q, P) == (raw + 255) // 256 * 256
+    assert L.mla_workspace_bytes(0, 1, 1, 1) == 0
+    assert L.mla_workspace_bytes(1, 1, 2000, 1) == 0   # rows above MLA_MAX_ROWS
+
+
+FAKE = 1 << 20  # a 256-aligned non-null address; never dereferenced (validation fails first)
+
+
+def _decode_call(L, **kw):
+    a = dict(q=FAKE, kv=FAKE, nblk=10, bt=FAKE, bts=4, sl=FAKE, tm=FAKE, ns=FAKE, P=4, b=2, s_q=1,
+             h_q=16, scale=0.1, causal=0, out=FAKE, lse=FAKE, ws=FAKE, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return L.mla_decode(a["q"], a["kv"], a["nblk"], a["bt"], a["bts"], a["sl"], a["tm"], a["ns"], a["P"],
+                        a["b"], a["s_q"], a["h_q"], a["scale"], a["causal"], a["out"], a["lse"], a["ws"],
+                        a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(q=None), dict(kv=None), dict(out=None), dict(ws=None), dict(q=FAKE + 8), dict(kv=FAKE + 2),
+    dict(ws=FAKE + 16), dict(b=0), dict(s_q=0), dict(h_q=0), dict(h_q=1025), dict(P=0), dict(nblk=0),
+    dict(bts=0), dict(scale=float("nan")), dict(scale=float("inf")), dict(causal=2),
+])
+def test_invalid_arguments_rejected_on_host(L, bad):
+    assert _decode_call(L, **bad) == 1  # MLA_ERR_INVALID_ARG
+
+
+def test_small_workspace_rejected_on_host(L):
+    assert _decode_call(L, wsb=1024) == 3  # MLA_ERR_WORKSPACE
+
+
+def test_metadata_argument_checks(L):
+    assert L.mla_get_metadata(None, 4, 16, 1, 4, 5, FAKE, FAKE, None) == 1
+    assert L.mla_get_metadata(FAKE, 4, 16, 1, 0, 5, FAKE, FAKE, None) == 1
+    assert L.mla_get_metadata(FAKE, 4, 16, 1, 4, -1, FAKE, FAKE, None) == 1
+    assert L.mla_get_metadata(FAKE + 2, 4, 16, 1, 4, 5, FAKE, FAKE, None) == 1
+
+
+def test_default_num_parts_argument_checks(L):
+    n = ctypes.c_int(0)
+    assert L.mla_default_num_parts(0, 0, 1, ctypes.byref(n)) == 1
+    assert L.mla_default_num_parts(0, 16, 1, None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        mla.get_metadata(torch.zeros(4, dtype=torch.int32), 16, 1, num_parts=4, fixed_cost=5)

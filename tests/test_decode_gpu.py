@@ -1,0 +1,122 @@
+"""GPU parity of the CUDA decode path against the CPU oracle (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import mla_decode_attention_14_b200 as mla
+import oracle
+from mla_decode_attention_14_b200 import workloads as W
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+
+
+def test_tiny_workload_full_parity():
+    wl = W.workload("tiny")
+    inp = W.make_inputs(wl, seed=0, tail="nan")
+    parity.full_parity(inp, what="tiny")
+
+
+SMALL = [
+    # seqlens, h_q, s_q, causal, num_parts
+    ([1, 63, 64, 65, 130, 257], 16, 1, False, None),
+    ([1, 63, 64, 65, 130, 257], 16, 1, False, 1),
+    ([1, 63, 64, 65, 130, 257], 16, 1, False, 7),
+    ([700, 5, 1290], 128, 1, False, None),
+    ([700, 5, 1290], 128, 1, False, 3),
+    ([129, 65, 1, 2, 200], 128, 2, True, None),     # 65 = 64k+1: query 0's last block is empty
+    ([129, 65, 1, 2, 200], 64, 2, True, 5),
+    ([3000, 17], 64, 1, False, 20),
+    ([64, 128, 192], 32, 1, False, 2),
+    ([513], 8, 2, False, 4),
+    ([33, 1000], 24, 3, True, 6),
+    ([250, 250, 250, 250], 128, 1, False, 74),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[str(i) for i in range(len(SMALL))])
+def test_small_shapes_parity(case):
+    seqlens, h_q, s_q, causal, parts = case
+    wl = W.custom(len(seqlens), h_q, s_q, seqlens, causal=causal)
+    inp = W.make_inputs(wl, seed=3, tail="nan", spare_blocks=2)
+    parity.full_parity(inp, num_parts=parts, what=str(case))
+
+
+@pytest.mark.parametrize("name", ["v2lite", "v3", "multitoken", "skewed"])
+def test_full_size_workloads_sampled_parity(name):
+    wl = W.workload(name)
+    inp = W.make_inputs(wl, seed=0, tail="nan")
+    out, lse, meta = parity.run_gpu(inp)
+    cum = meta.num_splits.cpu().numpy()
+    tasks = parity.sample_tasks(wl.seqlens, wl.s_q, wl.h_q, cum, np.random.default_rng(1))
+    ref_o, ref_l = oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
+                                 tasks=tasks)
+    o = parity.bf16_to_f64(out)
+    l = lse.cpu().numpy().astype(np.float64)
+    b, t, h = tasks[:, 0], tasks[:, 1], tasks[:, 2]
+    parity.compare(o[b, t, h], l[b, h, t], ref_o[b, t, h], ref_l[b, h, t], what=name)
+    # properties that hold for every row at any size
+    assert np.all(np.isfinite(o))
+    assert np.all(np.isfinite(l))
+
+
+def test_single_token_sequences_return_value_rows_exactly():
+    wl = W.custom(3, 128, 1, [1, 1, 1])
+    inp = W.make_inputs(wl, seed=5)
+    out, lse, _ = parity.run_gpu(inp)
+    kv = torch.from_numpy(inp["kv"]).view(torch.bfloat16)
+    for i in range(3):
+        v = kv[inp["block_table"][i, 0], 0, 0, :512]
+        assert torch.equal(out[i, 0].cpu(), v.expand(128, 512))
+
+
+def test_empty_sequences_give_zero_and_neg_inf():
+    wl = W.custom(3, 16, 2, [0, 70, 1], causal=True)
+    inp = W.make_inputs(wl, seed=6)
+    out, lse, _ = parity.full_parity(inp, what="empty")
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    assert torch.all(out[2, 0] == 0) and torch.all(torch.isneginf(lse[2, :, 0]))
+
+
+def test_deterministic():
+    wl = W.custom(4, 128, 1, [3000, 100, 4000, 65])
+    inp = W.make_inputs(wl, seed=7)
+    o1, l1, _ = parity.run_gpu(inp, num_parts=9)
+    o2, l2, _ = parity.run_gpu(inp, num_parts=9)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_bounds_violation_is_reported_not_faulted():
+    wl = W.custom(2, 16, 1, [100, 70])
+    inp = W.make_inputs(wl, seed=8)
+    inp["block_table"][1, 1] = inp["kv"].shape[0] + 5     # needed entry out of range
+    q, kv, bt, sl = parity.to_device(inp)
+    meta = mla.get_metadata(sl, 16, 1)
+    mla.decode(q, kv, bt, sl, inp["scale"], False, meta)
+    assert mla.check_status() == 6   # MLA_ERR_BOUNDS
+    assert mla.check_status() == 0   # cleared
+    # the library stays usable
+    inp2 = W.make_inputs(wl, seed=8)
+    parity.full_parity(inp2, what="after-bounds")
+
+
+def test_host_entry_point_matches_device_path():
+    wl = W.custom(3, 64, 2, [300, 1, 129], causal=True)
+    inp = W.make_inputs(wl, seed=9)
+    out_d, lse_d, _ = parity.run_gpu(inp)
+    dec = mla.HostDecoder(3, 2, 64, inp["kv"].shape[0], inp["block_table"].shape[1])
+    qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
+    kvh = torch.from_numpy(inp["kv"]).view(torch.bfloat16).pin_memory()
+    bth = torch.from_numpy(inp["block_table"]).pin_memory()
+    slh = torch.from_numpy(inp["seqlens"]).pin_memory()
+    oh = torch.empty((3, 2, 64, 512), dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty((3, 64, 2), dtype=torch.float32).pin_memory()
+    dec(qh, kvh, bth, slh, inp["scale"], True, oh, lh)
+    assert torch.equal(oh, out_d.cpu()) and torch.equal(lh, lse_d.cpu())
