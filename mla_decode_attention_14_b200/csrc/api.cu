@@ -4,6 +4,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
+
+#include <cuda.h>
 
 #include "../../include/mla.h"
 #include "common.cuh"
@@ -15,7 +18,8 @@ cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, in
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q,
                            __nv_bfloat16 *out, float *lse, const float *o_part,
                            const float *lse_part, cudaStream_t stream);
-cudaError_t launch_decode_simt(const DecodeParams &p, cudaStream_t stream);
+cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
+                                cudaStream_t stream);
 
 static std::atomic<int64_t> g_launches{0};
 
@@ -41,6 +45,73 @@ int check_device() {
         g_dev_ok[dev].store(st, std::memory_order_relaxed);
     }
     return st == 1 ? MLA_OK : MLA_ERR_UNSUPPORTED;
+}
+
+// ---- TMA descriptors of the paged cache, viewed as a 2-D bf16 tensor [num_blocks * 64, 576]:
+// "latent" boxes are 64 tokens x 64 dims with the 128-byte swizzle, "rope" boxes are
+// 64 tokens x 32 dims with the 64-byte swizzle (the layouts the MMA descriptors expect).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+struct MapEntry {
+    const void *kv;
+    int64_t num_blocks;
+    int device;
+    CUtensorMap lat, rope;
+};
+constexpr int kMapCache = 16;
+MapEntry g_maps[kMapCache];
+int g_maps_used = 0, g_maps_next = 0;
+std::mutex g_maps_mu;
+
+int cache_maps(const void *kv, int64_t num_blocks, CUtensorMap *lat, CUtensorMap *rope) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_maps_mu);
+    for (int k = 0; k < g_maps_used; ++k) {
+        if (g_maps[k].kv == kv && g_maps[k].num_blocks == num_blocks && g_maps[k].device == dev) {
+            *lat = g_maps[k].lat;
+            *rope = g_maps[k].rope;
+            return MLA_OK;
+        }
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    MapEntry e;
+    e.kv = kv;
+    e.num_blocks = num_blocks;
+    e.device = dev;
+    cuuint64_t dims[2] = {(cuuint64_t)MLA_D_QK, (cuuint64_t)num_blocks * MLA_BLOCK_TOKENS};
+    cuuint64_t strides[1] = {(cuuint64_t)MLA_D_QK * 2};
+    cuuint32_t box_lat[2] = {64, 64}, box_rope[2] = {32, 64}, estr[2] = {1, 1};
+    if (enc(&e.lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv), dims, strides, box_lat, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    if (enc(&e.rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv), dims, strides, box_rope, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    g_maps[g_maps_next] = e;
+    g_maps_next = (g_maps_next + 1) % kMapCache;
+    if (g_maps_used < kMapCache) ++g_maps_used;
+    *lat = e.lat;
+    *rope = e.rope;
+    return MLA_OK;
 }
 
 int shape_ok(int batch, int s_q, int h_q) {
@@ -180,7 +251,10 @@ int mla_decode_split(const void *q, const void *kv_cache, int64_t num_blocks,
     DecodeParams p = make_params(q, kv_cache, num_blocks, block_table, bt_stride, seqlens, tile_meta,
                                  num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
                                  workspace);
-    cudaError_t e = launch_decode_simt(p, static_cast<cudaStream_t>(stream));
+    CUtensorMap map_lat, map_rope;
+    rc = cache_maps(kv_cache, num_blocks, &map_lat, &map_rope);
+    if (rc != MLA_OK) return rc;
+    cudaError_t e = launch_decode_sm100(p, map_lat, map_rope, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

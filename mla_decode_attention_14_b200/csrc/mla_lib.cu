@@ -3,4 +3,4 @@
 #include "api.cu"
 #include "metadata.cu"
 #include "combine.cu"
-#include "decode_simt.cu"
+#include "decode_sm100.cu"
