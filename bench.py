@@ -178,42 +178,57 @@ def run_reference(args, wl, inp, counts):
 
 # --------------------------------------------------------------------------- our arm
 def cpu_baseline(wl, inp, target_s=12.0):
-    """The oracle, as it stands, on a bounded sample of the workload (rank 0, N = 1)."""
+    """The oracle, as it stands, on a bounded sample of the workload (rank 0, N = 1): whole
+    sequences (every query row, every key) in a seeded order until ~target_s of CPU work."""
     import oracle
     cores = os.cpu_count() or 1
-    seq = int(np.argsort(wl.seqlens)[len(wl.seqlens) // 2])   # a median-length sequence
-    n = int(wl.seqlens[seq])
+    order = np.random.default_rng(0).permutation(wl.batch)
+
+    def rows_of(seqs):
+        return np.array([[s, t, h] for s in seqs for t in range(wl.s_q) for h in range(wl.h_q)], np.int32)
+
     t0 = time.perf_counter()
     oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
-                  tasks=np.array([[seq, 0, 0]], np.int32), nthreads=1)
-    per_row = max(time.perf_counter() - t0, 1e-4)
-    nrows = int(max(cores, min(wl.rows, target_s * cores / per_row)))
-    tasks = np.array([[seq, (i // wl.h_q) % wl.s_q, i % wl.h_q] for i in range(nrows)], np.int32)
+                  tasks=rows_of([int(order[0])]), nthreads=cores)
+    per_token = max(time.perf_counter() - t0, 1e-6) / max(1, int(wl.seqlens[order[0]]))
+    chosen, est = [], 0.0
+    for s in order:
+        chosen.append(int(s))
+        est += per_token * max(1, int(wl.seqlens[s]))
+        if est >= target_s:
+            break
     t0 = time.perf_counter()
     oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
-                  tasks=tasks, nthreads=cores)
+                  tasks=rows_of(chosen), nthreads=cores)
     dt = time.perf_counter() - t0
-    # the metric's unit: algorithmic bytes (the sequence's KV once + sampled q rows) per second
-    val = (n * 1152 + nrows * 1152) / dt / 1e12
+    n = int(sum(int(wl.seqlens[s]) for s in chosen))
+    # the metric's unit: algorithmic bytes (each sampled sequence's KV once + its query rows) per second
+    val = (n * 1152 + len(chosen) * wl.rows * 1152) / dt / 1e12
     return {"value": val, "unit": "TB/s", "cores": cores, "kind": "oracle",
-            "sample": "%d of %d query rows of one %d-token sequence (all its keys), %.1f s" % (nrows, wl.rows, n, dt),
+            "sample": "%d of %d sequences (%d tokens, all %d query rows each), %.1f s on %d threads"
+                      % (len(chosen), wl.batch, n, wl.rows, dt, cores),
             "seconds": dt}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="v3", choices=W.NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--max-batch", type=int, default=0,
+                    help="keep only the first N sequences (for profiler captures of a smaller slice)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     wl = W.workload(args.workload)
+    if args.max_batch and args.max_batch < wl.batch:
+        wl = W.custom(args.max_batch, wl.h_q, wl.s_q, wl.seqlens[:args.max_batch], wl.causal, wl.scale,
+                      name="%s[:%d]" % (wl.name, args.max_batch))
     counts = W.algorithmic_counts(wl)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

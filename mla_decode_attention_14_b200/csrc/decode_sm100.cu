@@ -1,8 +1,8 @@
 // decode_sm100.cu -- the B200 (sm_100a) split kernel of MLA decode attention.
 //
 // What it computes (per query row r of sequence b, over that sequence's visible keys j):
-// S_j = scale * <q_r, k_j> over all 576 latent+rotary dims ("Gemm1"), an fp32 online softmax,
-// and O = sum_j softmax_j * k_j[0:512] ("Gemm2"). "Deep analysis of the DeepSeek Infra
+// S_j = scale * <q_r, k_j> over all 576 latent+rotary dims ("Gemm1"), an online softmax in
+// fp32, and O = sum_j softmax_j * k_j[0:512] ("Gemm2"). "Deep analysis of the DeepSeek Infra
 // open-source releases" (jingzhunhuoke.net/55333.html), DAY1 FlashMLA: the cache is kept in
 // 64-token blocks (feature (2)), the kernel streams each block once and runs Gemm1 then Gemm2
 // on it (feature (4)), and lengths are load-balanced over the SMs (feature (5)).
@@ -12,27 +12,39 @@
 //    The fp32 accumulator O for 128 rows x 512 value dims is 256 KB -- all of one SM's tensor
 //    memory -- so each CTA of the pair owns HALF of the value dims (O: 128 lanes x 256 columns
 //    of TMEM) and streams only the cache columns it needs: CTA h loads latent dims
-//    [256h, 256h+256) and rotary dims [512+32h, 512+32h+32), i.e. exactly half of every
-//    block (36,864 bytes); the pair together reads each block once.
+//    [256h, 256h+256) and rotary dims [512+32h, 512+32h+32), i.e. exactly half of every block
+//    (36,864 bytes); the pair together reads each block once.
 //  * Gemm1 is split along its 576-long contraction: CTA h computes the partial scores over its
-//    288 dims (18 tcgen05 MMAs, M=128 rows, N=64 tokens, K=16, A = this half of Q held in
-//    TMEM, B = the K tile in shared memory). The two partial score tiles (128 x 64 fp32) are
-//    swapped through distributed shared memory (st.async completing on the receiver's
-//    mbarrier); both CTAs add them in the same order and so hold bit-identical scores.
-//  * Softmax warps (one thread per query row = one TMEM lane) apply the scale, masks (tail
-//    and causal), an online max with lazy rescaling (O is rescaled only when the running max
-//    grows by more than 2^8), write P (bf16) into TMEM and release Gemm2.
-//  * Gemm2: 4 MMAs (M=128, N=256, K=16 tokens each) with A = P from TMEM and B = the value
-//    half of the same shared-memory tile read MN-major -- the block is loaded once for both
-//    GEMMs.
+//    288 dims (18 tcgen05 MMAs, M=128 rows, N=64 tokens; the latent part of Q is the A operand
+//    in TMEM, the rotary part in shared memory).
+//  * The pair combines the partial scores multiplicatively: 2^(s0 + s1 - m) =
+//    2^(s0 - m0) * 2^(s1 - m1) * 2^(m0 + m1 - m). Each CTA computes E = 2^(s - m) for its own
+//    partial with its own row offset m, keeps it in fp32, and sends it to the peer as fp16
+//    (scaled by 2^15) together with m in fp32: st.async stores into the peer's 2-slot receive
+//    ring complete on the peer's mbarrier. The relative error of the exchanged factor is that
+//    of fp16 (2^-11) whatever the score magnitude, and the traffic is half that of fp32 scores.
+//  * Eight softmax warps: warp w serves TMEM lane quarter w&3 (32 query rows) and one half of
+//    every block's tokens; the two halves of a row agree on an upper bound of the block max
+//    through shared memory, so both take the same lazy-rescaling decisions (O is rescaled only
+//    when the running max grows by more than 2^8). P = E_own * E_peer * 2^(m0 + m1 - m) goes
+//    to TMEM as two bf16 terms, hi = bf16(P) and lo = bf16(P - hi), so P's rounding does not
+//    add to the bf16 output rounding.
+//  * Issuing a tcgen05 MMA blocks the issuing thread until the tensor core takes it, so the MMA
+//    warp's program order is the tensor-core schedule: Gemm1 of block g+1 runs while the softmax
+//    warps finish block g, Gemm2 of block g right after.
+//  * Gemm2: 8 MMAs (M=128, N=256, K=16 tokens; A = P_hi then P_lo from TMEM, B = the value half
+//    of the same shared-memory tile read MN-major): the block is loaded once for both GEMMs.
 //  * Warp roles: warp 0 lane 0 = TMA producer (4-stage ring, block-table gather, L2
 //    evict-first); warp 1 = MMA warp (lane 0 issues; the warp owns the TMEM allocation and
 //    zeroes the cache rows past a sequence's end before any MMA reads them, so undefined
-//    tail contents never reach the result); warps 4-7 = softmax, correction and epilogue
-//    (warps 2-3 idle: the softmax warps must sit in TMEM lane quarters 0-3).
+//    tail contents never reach the result); warps 4-11 = softmax, correction and epilogue
+//    (warps 2-3 idle: the softmax warps must start at a multiple of 4 so that warp w serves
+//    TMEM lane quarter w & 3).
 //  * Pieces of split sequences leave fp32 partial O and lse in the workspace for the combine
 //    kernel; whole sequences are written straight to bf16 out / fp32 lse.
 // Every wait is bounded; a timeout sets the device error word and the CTA exits cleanly.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -41,26 +53,33 @@ using namespace sm100;
 
 namespace dec {
 constexpr int kStages = 4;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kBoxBytes = kBlk * 128;                      // 64 tokens x 64 bf16 (128-byte swizzle)
 constexpr int kRopeBoxBytes = kBlk * 64;                   // 64 tokens x 32 bf16 (64-byte swizzle)
 constexpr int kStageBytes = 4 * kBoxBytes + kRopeBoxBytes;  // 36,864: half of one cache block
-constexpr int kXchgFloats = 128 * 64;                      // partial score tile of one block
 constexpr float kRescaleThreshold = 8.0f;                  // log2 units: rescale O when max grows > 2^8
+// The peer's factors E = 2^(s - m) <= 1 cross the cluster as fp16 scaled by 2^15 (< 65504), which
+// keeps values down to 2^-29 normal (full 11-bit precision); the receiver folds 2^-15 back in.
+constexpr float kXScale = 32768.0f;
+constexpr float kXScaleLog2 = 15.0f;
 
 // TMEM column map (512 columns allocated, 128 lanes = 128 query rows)
-constexpr uint32_t kTmemO = 0;    // 256 fp32: O for this CTA's 256 value dims
-constexpr uint32_t kTmemS = 256;  // 64 fp32: partial scores of the current block
-constexpr uint32_t kTmemQ = 320;  // 144 x (2 bf16): this CTA's 288 query dims
-constexpr uint32_t kTmemP = 464;  // 32 x (2 bf16): probabilities of the current block
+constexpr uint32_t kTmemO = 0;     // 256 fp32: O for this CTA's 256 value dims
+constexpr uint32_t kTmemQ = 256;   // 128 x (2 bf16): this CTA's 256 latent query dims
+constexpr uint32_t kTmemS = 384;   // 64 fp32: partial scores of the current block
+constexpr uint32_t kTmemPhi = 448; // 32 x (2 bf16): P rounded to bf16
+constexpr uint32_t kTmemPlo = 480; // 32 x (2 bf16): bf16 of P's rounding residue
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(1024) Smem {
-    uint8_t stage[kStages][kStageBytes];
-    float4 xchg[2][16][128];  // [slot][4-column group][row]: partial scores written by the peer CTA
+    uint8_t stage[kStages][kStageBytes];  // KV ring
+    uint4 xchg[2 * 2 * 4 * 128 + 2 * 2 * 128 / 4];  // peer E factors (fp16) [slot][token half][16 B][row]
+                                                    // + row offsets (fp32) [slot][token half][row]
+    float xmax[2][2][128], xsum[2][128];            // per-row exchange between the two token halves
+    uint8_t q_rope[128 * 64];             // rotary query dims [128 rows x 32], K-major, 64-byte swizzle
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full, s_free, p_full, p_free, o_full, o_free, q_full, mma_done;
-    uint64_t xfull[2];
+    uint64_t xfull[2];  // receive slots filled by the peer
     uint32_t tmem_base;
     int abort;
 };
@@ -102,39 +121,59 @@ struct Cursor {
     }
 };
 
-__device__ __forceinline__ bool is_tail_block(const Piece &pc, int blk) {
-    return blk == num_blocks_of(pc.n) - 1 && (pc.n % kBlk) != 0;
-}
+// Walks the blocks of one part in order, with piece boundaries.
+struct BlockWalker {
+    Cursor cur;
+    Piece pc;
+    int blk, piece_k;
+    bool live;
+    __device__ void init(const int32_t *meta, const DecodeParams &p) {
+        cur.init(meta, p.batch);
+        live = cur.next(p, pc);
+        blk = live ? pc.lo : 0;
+        piece_k = 0;
+    }
+    __device__ bool first() const { return blk == pc.lo; }
+    __device__ bool last() const { return blk == pc.hi - 1; }
+    __device__ bool tail() const { return blk == num_blocks_of(pc.n) - 1 && (pc.n % kBlk) != 0; }
+    __device__ void advance(const DecodeParams &p) {
+        if (blk + 1 < pc.hi) {
+            ++blk;
+            return;
+        }
+        live = cur.next(p, pc);
+        if (live) {
+            blk = pc.lo;
+            ++piece_k;
+        }
+    }
+};
 
 // ---------------------------------------------------------------- TMA producer (1 thread)
 __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map_lat, const CUtensorMap *map_rope,
                          const int32_t *meta, uint32_t half) {
     const uint64_t policy = l2_evict_first_policy();
-    Cursor cur;
-    cur.init(meta, p.batch);
-    Piece pc;
+    BlockWalker w;
+    w.init(meta, p);
     int gidx = 0;
     bool bad_block = false;
-    while (cur.next(p, pc)) {
-        for (int blk = pc.lo; blk < pc.hi; ++blk, ++gidx) {
-            const int s = gidx % kStages, fill = gidx / kStages;
-            if (fill > 0 && !mbar_wait(&sm.kv_empty[s], (fill - 1) & 1, &sm.abort)) goto drain;
-            const int phys = blk < p.bt_stride ? __ldg(&p.block_table[(size_t)pc.seq * p.bt_stride + blk]) : -1;
-            if (phys < 0 || (int64_t)phys >= p.num_blocks) {
-                bad_block = true;
-                mbar_arrive(&sm.kv_full[s]);  // consumers run on stale data; the error word reports it
-                continue;
-            }
-            mbar_arrive_expect_tx(&sm.kv_full[s], kStageBytes);
-            const int y = phys * kBlk;
-            uint8_t *dst = sm.stage[s];
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-                tma_load_2d(dst + b * kBoxBytes, map_lat, 256 * (int)half + 64 * b, y, &sm.kv_full[s], policy);
-            tma_load_2d(dst + 4 * kBoxBytes, map_rope, 512 + 32 * (int)half, y, &sm.kv_full[s], policy);
+    for (; w.live; w.advance(p), ++gidx) {
+        const int s = gidx % kStages, fill = gidx / kStages;
+        if (fill > 0 && !mbar_wait(&sm.kv_empty[s], (fill - 1) & 1, &sm.abort)) break;
+        const int phys = w.blk < p.bt_stride ? __ldg(&p.block_table[(size_t)w.pc.seq * p.bt_stride + w.blk]) : -1;
+        if (phys < 0 || (int64_t)phys >= p.num_blocks) {
+            bad_block = true;
+            mbar_arrive(&sm.kv_full[s]);  // consumers run on stale data; the error word reports it
+            continue;
         }
+        mbar_arrive_expect_tx(&sm.kv_full[s], kStageBytes);
+        const int y = phys * kBlk;
+        uint8_t *dst = sm.stage[s];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            tma_load_2d(dst + b * kBoxBytes, map_lat, 256 * (int)half + 64 * b, y, &sm.kv_full[s], policy);
+        tma_load_2d(dst + 4 * kBoxBytes, map_rope, 512 + 32 * (int)half, y, &sm.kv_full[s], policy);
     }
-drain:
     if (bad_block) raise_error(kErrBounds);
     // every load still in flight must land before the CTA may exit
     for (int k = max(0, gidx - kStages); k < gidx; ++k) {
@@ -145,15 +184,14 @@ drain:
 }
 
 // ---------------------------------------------------------------- MMA warp
-// Lane 0 waits on the barriers and issues every tcgen05 MMA/commit; the whole warp zeroes
-// the cache rows past a sequence's end in that sequence's last block (undefined contents --
-// possibly NaN -- must not reach Gemm2 even with zero probabilities) before lane 0 issues.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int lane) {
     bool ok = true;
     if (lane == 0) ok = mbar_wait(bar, parity, abort);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Zero the cache rows past a sequence's end in its last block (undefined contents -- possibly
+// NaN -- must not reach Gemm2 even with zero probabilities).
 __device__ void zero_tail_rows(uint8_t *st, int valid, int lane) {
     const int zr = kBlk - valid;
     const uint4 z = make_uint4(0, 0, 0, 0);
@@ -171,58 +209,63 @@ __device__ void mma_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, u
     constexpr uint32_t id1 = idesc_bf16_f32(128, 64, 0);   // S = Q K^T: K-major B
     constexpr uint32_t id2 = idesc_bf16_f32(128, 256, 1);  // O += P V: MN-major B
     const int lane = threadIdx.x & 31;
-    Cursor cur;
-    cur.init(meta, p.batch);
-    Piece pc;
-    int gidx = 0, piece_k = 0;
     volatile int *abort = &sm.abort;
+    BlockWalker w1, w2;  // w1: next Gemm1, w2: next Gemm2 (one block behind)
+    w1.init(meta, p);
+    w2 = w1;
+    int g1 = 0, g2 = 0;
 
-    // O += P_b V_b for block b (global index); first == first block of its piece
-    auto gemm2 = [&](int b, bool first) -> bool {
-        if (!warp_wait(&sm.p_full, b & 1, abort, lane)) return false;
-        if (first && piece_k > 0 && !warp_wait(&sm.o_free, (piece_k - 1) & 1, abort, lane)) return false;
+    // Gemm1 of block g1 into S_a / S_b (two interleaved accumulation chains)
+    auto gemm1 = [&]() -> bool {
+        if (w1.first() && !warp_wait(&sm.q_full, w1.piece_k & 1, abort, lane)) return false;
+        const int s = g1 % kStages;
+        if (!warp_wait(&sm.kv_full[s], (g1 / kStages) & 1, abort, lane)) return false;
+        if (w1.tail()) zero_tail_rows(sm.stage[s], w1.pc.n - w1.blk * kBlk, lane);
+        if (g1 > 0 && !warp_wait(&sm.s_free, (g1 - 1) & 1, abort, lane)) return false;
         if (lane == 0) {
             tc_fence_after();
-            const uint32_t st = smem_addr(sm.stage[b % kStages]);
+            // descriptors: one base each, then constant offsets (address field is in 16-byte units)
+            const uint64_t kd = smem_desc(smem_addr(sm.stage[s]), 16, 1024, 2);
+            const uint64_t rd = smem_desc(smem_addr(sm.stage[s]) + 4 * kBoxBytes, 16, 512, 4);
+            const uint64_t qd = smem_desc(smem_addr(sm.q_rope), 16, 512, 4);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, smem_desc(st + kk * 2048, 4 * 2048, 1024, 2), id2,
-                       (!first || kk > 0) ? 1u : 0u);
-            mma_commit(&sm.p_free);
-            mma_commit(&sm.kv_empty[b % kStages]);
+            for (int k = 0; k < 16; ++k)  // latent k-steps, A (Q) from TMEM
+                mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * k,
+                       kd + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id1, k > 0 ? 1u : 0u);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)  // rotary k-steps, A from shared memory
+                mma_ss(tmem + kTmemS, qd + 2 * c, rd + 2 * c, id1, 1u);
+            mma_commit(&sm.s_full);
         }
         __syncwarp();
+        ++g1;
+        w1.advance(p);
         return true;
     };
 
-    while (cur.next(p, pc)) {
-        if (!warp_wait(&sm.q_full, piece_k & 1, abort, lane)) goto done;
-        {
-            const int nb = pc.hi - pc.lo;
-            for (int j = 0; j < nb; ++j, ++gidx) {
-                const int s = gidx % kStages;
-                if (!warp_wait(&sm.kv_full[s], (gidx / kStages) & 1, abort, lane)) goto done;
-                if (is_tail_block(pc, pc.lo + j)) zero_tail_rows(sm.stage[s], pc.n - (pc.lo + j) * kBlk, lane);
-                if (gidx > 0 && !warp_wait(&sm.s_free, (gidx - 1) & 1, abort, lane)) goto done;
-                if (lane == 0) {
-                    tc_fence_after();
-                    const uint32_t st = smem_addr(sm.stage[s]);
+    if (w1.live && !gemm1()) goto done;
+    while (w2.live) {
+        if (w1.live && !gemm1()) goto done;
+        // Gemm2 of block g2: O (+)= P V
+        if (!warp_wait(&sm.p_full, g2 & 1, abort, lane)) goto done;
+        if (w2.first() && w2.piece_k > 0 && !warp_wait(&sm.o_free, (w2.piece_k - 1) & 1, abort, lane)) goto done;
+        if (lane == 0) {
+            tc_fence_after();
+            const uint64_t vd = smem_desc(smem_addr(sm.stage[g2 % kStages]), 4 * 2048, 1024, 2);
+            const bool first = w2.first();
 #pragma unroll
-                    for (int k = 0; k < 18; ++k) {
-                        const uint64_t bd = k < 16 ? smem_desc(st + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024, 2)
-                                                   : smem_desc(st + 4 * kBoxBytes + (k - 16) * 32, 16, 512, 4);
-                        mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * k, bd, id1, k > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm.s_full);
-                }
-                __syncwarp();
-                if (j > 0 && !gemm2(gidx - 1, j == 1)) goto done;
-            }
-            if (!gemm2(gidx - 1, nb == 1)) goto done;
-            if (lane == 0) mma_commit(&sm.o_full);
-            __syncwarp();
-            ++piece_k;
+            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo: O += (P_hi + P_lo) V, A from TMEM
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tmem + kTmemO, tmem + (hl ? kTmemPlo : kTmemPhi) + 8 * kk, vd + 128 * kk, id2,
+                           (!first || hl > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&sm.p_free);
+            mma_commit(&sm.kv_empty[g2 % kStages]);
+            if (w2.last()) mma_commit(&sm.o_full);
         }
+        __syncwarp();
+        ++g2;
+        w2.advance(p);
     }
 done:
     // all issued MMAs complete before teardown (bounded; independent of the abort flag)
@@ -235,209 +278,295 @@ done:
     __syncwarp();
 }
 
-// ---------------------------------------------------------------- softmax / epilogue (warps 4-7)
-__device__ __forceinline__ void load_q(const DecodeParams &p, const Piece &pc, int r, bool row_ok, uint32_t half,
-                                       uint32_t taddr) {
-    const uint4 *qrow = reinterpret_cast<const uint4 *>(p.q + ((size_t)pc.seq * p.rows + (row_ok ? r : 0)) * kDqk);
+// ---------------------------------------------------------------- softmax / epilogue (warps 4-11)
+// Eight warps: warp w handles TMEM lane quarter (w & 3) -- 32 query rows -- and token half
+// th = (w - 4) >> 2 of every block (tokens [32 th, 32 th + 32)); for O it owns columns
+// [128 th, 128 th + 128). One thread = one (row, token half).
+struct SoftCtx {
+    const DecodeParams *p;
+    uint32_t tmem, lane_off, half, xchg_peer, xfull_peer0;
+    int i, lane, r, th;
+    bool row_ok, warp_ok;
+};
+
+// Q of piece `pc`: latent half -> TMEM (this warp's lanes, its 64 of the 128 columns),
+// rotary half -> shared memory (its 2 of the 4 chunks of the row).
+__device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &pc) {
+    if (c.warp_ok) {
+        const DecodeParams &p = *c.p;
+        const uint4 *qrow =
+            reinterpret_cast<const uint4 *>(p.q + ((size_t)pc.seq * p.rows + (c.row_ok ? c.r : 0)) * kDqk);
 #pragma unroll 1
-    for (int c16 = 0; c16 < 9; ++c16) {  // 9 x 16 columns = 288 bf16 (256 latent + 32 rotary)
-        uint32_t w[16];
-        const int off = c16 < 8 ? (256 * (int)half + 32 * c16) / 8 : (512 + 32 * (int)half) / 8;
+        for (int c16 = 4 * c.th; c16 < 4 * c.th + 4; ++c16) {  // 16 columns = 32 latent bf16 each
+            uint32_t w[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const uint4 x = row_ok ? __ldg(qrow + off + v) : make_uint4(0, 0, 0, 0);
-            w[4 * v + 0] = x.x;
-            w[4 * v + 1] = x.y;
-            w[4 * v + 2] = x.z;
-            w[4 * v + 3] = x.w;
+            for (int v = 0; v < 4; ++v) {
+                const uint4 x = c.row_ok ? __ldg(qrow + (256 * (int)c.half + 32 * c16) / 8 + v) : make_uint4(0, 0, 0, 0);
+                w[4 * v + 0] = x.x;
+                w[4 * v + 1] = x.y;
+                w[4 * v + 2] = x.z;
+                w[4 * v + 3] = x.w;
+            }
+            tmem_st16(c.tmem + kTmemQ + c.lane_off + 16 * c16, w);
         }
-        tmem_st16(taddr + 16 * c16, w);
+#pragma unroll
+        for (int v = 2 * c.th; v < 2 * c.th + 2; ++v) {  // rotary dims: 16-byte chunks, 64-byte swizzle
+            const uint4 x = c.row_ok ? __ldg(qrow + (512 + 32 * (int)c.half) / 8 + v) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sm.q_rope + c.i * 64 + ((v ^ ((c.i >> 1) & 3)) * 16)) = x;
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
     }
-    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&sm.q_full);
+}
+
+// Own partial scores of block g for this thread's 32 tokens: S_a + S_b (log2 units), then
+// E = 2^(s - m) with m the thread's own max; frees the accumulators and sends E (fp16) and m
+// (fp32) to the peer CTA's receive slot g % 2.
+__device__ __forceinline__ bool load_and_send(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&e)[32],
+                                              float &m_own) {
+    if (!mbar_wait(&sm.s_full, g & 1, &sm.abort)) return false;
+    tc_fence_after();
+    m_own = -INFINITY;
+    if (c.warp_ok) {
+        uint32_t a[32];
+        tmem_ld32(c.tmem + kTmemS + c.lane_off + 32 * c.th, a);
+        tmem_wait_ld();
+        const float sl2 = c.p->scale_log2;
+        const int k0 = key0 + 32 * c.th;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float v = __uint_as_float(a[j]) * sl2;
+            e[j] = k0 + j < vis ? v : -INFINITY;
+        }
+        float t[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) t[j] = fmaxf(e[j], e[j + 16]);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+            for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+        m_own = t[0];
+        const bool none = m_own == -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) e[j] = none ? 0.f : ex2_approx(e[j] - m_own);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&sm.s_free);
+    if (c.warp_ok) {
+        const int slot = g & 1;
+        const uint32_t base = c.xchg_peer + (uint32_t)(((slot * 2 + c.th) * 4) * 128 + c.i) * 16;
+        const uint32_t bar = c.xfull_peer0 + slot * 8;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                __half2 two = __floats2half2_rn(e[8 * c4 + 2 * q] * kXScale, e[8 * c4 + 2 * q + 1] * kXScale);
+                w[q] = *reinterpret_cast<uint32_t *>(&two);
+            }
+            st_async_v4_b32(base + c4 * 128 * 16, w[0], w[1], w[2], w[3], bar);
+        }
+        // the row offset travels in the offsets area of the same slot
+        const uint32_t off = c.xchg_peer + (uint32_t)(2 * 2 * 4 * 128 * 16) + (uint32_t)((slot * 2 + c.th) * 128 + c.i) * 4;
+        st_async_b32(off, __float_as_uint(m_own), bar);
+    }
+    return true;
 }
 
 __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem, uint32_t half,
                              int group) {
-    const int i = threadIdx.x - 128;  // row within the group == TMEM lane
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    SoftCtx c;
+    c.p = &p;
+    c.tmem = tmem;
+    c.half = half;
+    const int warp = threadIdx.x >> 5;
     const int wq = warp & 3;
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int r = group * 128 + i;
-    const bool row_ok = r < p.rows;
-    const bool warp_ok = group * 128 + wq * 32 < p.rows;
-    const int nvalid_warps = min(4, (p.rows - group * 128 + 31) / 32);
-    const uint32_t xbytes = (uint32_t)nvalid_warps * 32 * 16 * 16;
-    const int t_q = row_ok ? r / p.h_q : 0, h_idx = row_ok ? r % p.h_q : 0;
+    c.th = (warp - 4) >> 2;
+    c.lane = threadIdx.x & 31;
+    c.i = wq * 32 + c.lane;  // row within the group == TMEM lane
+    c.lane_off = (uint32_t)(wq * 32) << 16;
+    c.r = group * 128 + c.i;
+    c.row_ok = c.r < p.rows;
+    c.warp_ok = group * 128 + wq * 32 < p.rows;
     const uint32_t peer = half ^ 1u;
-    const uint32_t xchg_peer = map_to_rank(&sm.xchg[0][0][0], peer);
-    const uint32_t xfull_peer0 = map_to_rank(&sm.xfull[0], peer);
+    c.xchg_peer = map_to_rank(&sm.xchg[0], peer);
+    c.xfull_peer0 = map_to_rank(&sm.xfull[0], peer);
+    const int nvalid_warps = min(4, (p.rows - group * 128 + 31) / 32);
+    const uint32_t xbytes = (uint32_t)nvalid_warps * 2 * 32 * (64 + 4);  // both token halves: E (64 B) + offset
+    const int t_q = c.row_ok ? c.r / p.h_q : 0, h_idx = c.row_ok ? c.r % p.h_q : 0;
     volatile int *abort = &sm.abort;
-    const float sl2 = p.scale_log2;
+    const float4 *xe = reinterpret_cast<const float4 *>(sm.xchg);
+    const float *xo = reinterpret_cast<const float *>(sm.xchg + 2 * 2 * 4 * 128);  // offsets area
 
-    Cursor cur;
-    cur.init(meta, p.batch);
-    Piece pc;
-    bool have = cur.next(p, pc);
-    if (have) {
-        if (warp_ok) load_q(p, pc, r, row_ok, half, tmem + kTmemQ + lane_off);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.q_full);
+    BlockWalker wa;
+    wa.init(meta, p);
+    if (!wa.live) return;
+    load_q(sm, c, wa.pc);
+    int vis = c.row_ok ? visible_keys(wa.pc.n, p.s_q, t_q, p.causal) : 0;
+    float e_own[32], m_own;
+    if (!load_and_send(sm, c, 0, wa.blk * kBlk, vis, e_own, m_own)) return;
+    if (wa.last()) {  // the next piece's Q may replace this one once its last Gemm1 is done
+        Cursor tmp = wa.cur;
+        Piece nx;
+        if (tmp.next(p, nx)) load_q(sm, c, nx);
     }
-    int gidx = 0, piece_k = 0;
-    while (have) {
-        const Piece cp = pc;
-        const int vis = row_ok ? visible_keys(cp.n, p.s_q, t_q, p.causal) : 0;
-        float m_ref = -INFINITY, l = 0.f;
-        const int nb = cp.hi - cp.lo;
-        for (int j = 0; j < nb; ++j, ++gidx) {
-            const int slot = gidx & 1;
-            if (threadIdx.x == 128) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
-            if (!mbar_wait(&sm.s_full, gidx & 1, abort)) return;
-            tc_fence_after();
-            uint32_t sv[64];
-            if (warp_ok) {
-                uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-                uint32_t (&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-                tmem_ld32(tmem + kTmemS + lane_off, a);
-                tmem_ld32(tmem + kTmemS + lane_off + 32, b);
-                tmem_wait_ld();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_free);
-            // swap partial scores with the peer CTA
-            if (warp_ok) {
-                const uint32_t dst = xchg_peer + (uint32_t)((slot * 16) * 128 + i) * 16;
-                const uint32_t bar = xfull_peer0 + slot * 8;
+    float m_ref = -INFINITY, l = 0.f;
+    for (int g = 0; wa.live; ++g) {
+        BlockWalker wb = wa;
+        wb.advance(p);
+        // peer factors of block g (slot g % 2)
+        const int slot = g & 1;
+        if (threadIdx.x == 128) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
+        if (!mbar_wait_cluster(&sm.xfull[slot], (g >> 1) & 1, abort)) return;
+        float e_peer[32];
+        float m_peer = -INFINITY;
+        if (c.warp_ok) {
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4)
-                    st_async_v4(dst + c4 * 128 * 16, __uint_as_float(sv[4 * c4]), __uint_as_float(sv[4 * c4 + 1]),
-                                __uint_as_float(sv[4 * c4 + 2]), __uint_as_float(sv[4 * c4 + 3]), bar);
-            }
-            if (!mbar_wait_cluster(&sm.xfull[slot], (gidx >> 1) & 1, abort)) return;
-            bool need = false;
-            float alpha = 1.f;
-            uint32_t pk[32];
-            if (warp_ok) {
-                const int key0 = (cp.lo + j) * kBlk;
-                float s[64];
-                float mb = -INFINITY;
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 v = xe[((slot * 2 + c.th) * 4 + c4) * 128 + c.i];
+                const uint32_t w[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+                                       __float_as_uint(v.w)};
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4) {
-                    const float4 o = sm.xchg[slot][c4][i];
-                    const float po[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 4 * c4 + e;
-                        const float v = (__uint_as_float(sv[c]) + po[e]) * sl2;
-                        s[c] = key0 + c < vis ? v : -INFINITY;
-                        mb = fmaxf(mb, s[c]);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[q]));
+                    e_peer[8 * c4 + 2 * q] = f.x;
+                    e_peer[8 * c4 + 2 * q + 1] = f.y;
                 }
-                if (j == 0) {
-                    m_ref = mb;
-                } else if (mb > m_ref + kRescaleThreshold) {
-                    if (m_ref == -INFINITY) {
-                        m_ref = mb;  // nothing accumulated yet (O and l are zero)
-                    } else {
-                        alpha = exp2f(m_ref - mb);
-                        m_ref = mb;
-                        l *= alpha;
-                        need = true;
-                    }
-                }
-                float sum = 0.f;
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float p0 = m_ref == -INFINITY ? 0.f : exp2f(s[c] - m_ref);
-                    const float p1 = m_ref == -INFINITY ? 0.f : exp2f(s[c + 1] - m_ref);
-                    sum += p0 + p1;
-                    __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
-                    pk[c >> 1] = *reinterpret_cast<uint32_t *>(&two);
-                }
-                l += sum;
             }
-            // P buffer and O are free once Gemm2 of the previous block has completed
-            if (gidx > 0 && !mbar_wait(&sm.p_free, (gidx - 1) & 1, abort)) return;
-            tc_fence_after();
-            if (warp_ok) {
-                if (__any_sync(0xffffffffu, need)) {
-                    const float a = need ? alpha : 1.f;
+            m_peer = xo[(slot * 2 + c.th) * 128 + c.i];
+        }
+        // an upper bound of the block's row max (both token halves), shared by the two warps of a row
+        const float mbu_half = m_own + m_peer;
+        sm.xmax[g & 1][c.th][c.i] = mbu_half;
+        named_bar_sync(1, 256);
+        const float mbu = fmaxf(mbu_half, sm.xmax[g & 1][c.th ^ 1][c.i]);
+        bool need = false;
+        float alpha = 1.f;
+        if (wa.first()) {
+            m_ref = mbu;
+            l = 0.f;
+        } else if (mbu > m_ref + kRescaleThreshold) {
+            if (m_ref == -INFINITY) {
+                m_ref = mbu;  // nothing accumulated yet (O and l are zero)
+            } else {
+                alpha = ex2_approx(m_ref - mbu);
+                m_ref = mbu;
+                l *= alpha;
+                need = true;
+            }
+        }
+        uint32_t pk[16], pl[16];  // P rounded to bf16 (hi) and the bf16 of its rounding residue (lo)
+        if (c.warp_ok) {
+            const bool none = m_ref == -INFINITY || mbu_half == -INFINITY;
+            const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - kXScaleLog2);
+            float su[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                const float p0 = e_own[j] * e_peer[j] * f, p1 = e_own[j + 1] * e_peer[j + 1] * f;
+                su[(j >> 1) & 3] += p0 + p1;
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+                const float2 hf = __bfloat1622float2(hi);
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&hi);
+                pl[j >> 1] = *reinterpret_cast<const uint32_t *>(&lo);
+            }
+            l += (su[0] + su[1]) + (su[2] + su[3]);
+        }
+        // the P tile and O are free once Gemm2 of block g-1 has completed
+        if (g > 0 && !mbar_wait(&sm.p_free, (g - 1) & 1, abort)) return;
+        tc_fence_after();
+        if (c.warp_ok) {
+            if (__any_sync(0xffffffffu, need)) {
+                const float a = need ? alpha : 1.f;
 #pragma unroll 1
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + kTmemO + lane_off + 32 * c, v);
-                        tmem_wait_ld();
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + kTmemO + c.lane_off + 128 * c.th + 32 * q, v);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * a);
-                        tmem_st32(tmem + kTmemO + lane_off + 32 * c, v);
-                    }
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * a);
+                    tmem_st32(tmem + kTmemO + c.lane_off + 128 * c.th + 32 * q, v);
                 }
-                tmem_st32(tmem + kTmemP + lane_off, pk);
                 tmem_wait_st();
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full);
-        }
-        // the last Gemm1 of this piece has completed: Q may be replaced by the next piece's
-        have = cur.next(p, pc);
-        if (have) {
-            if (warp_ok) load_q(p, pc, r, row_ok, half, tmem + kTmemQ + lane_off);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.q_full);
-        }
-        // epilogue of piece cp
-        if (!mbar_wait(&sm.o_full, piece_k & 1, abort)) return;
-        tc_fence_after();
-        if (warp_ok) {
-            const bool empty = !(l > 0.f);
-            const float inv = empty ? 0.f : 1.f / l;
-            const float lse = empty ? -INFINITY : (m_ref + log2f(l)) * 0.69314718055994530942f;
-            const bool whole = cp.nsplit == 1;
-#pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tmem + kTmemO + lane_off + 32 * c, v);
-                tmem_wait_ld();
-                if (!row_ok) continue;
-                if (whole) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)cp.seq * p.rows + r) * kDv +
-                                                           256 * half + 32 * c);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(v[8 * q4 + 2 * e]) * inv,
-                                                                       __uint_as_float(v[8 * q4 + 2 * e + 1]) * inv);
-                            w[e] = *reinterpret_cast<uint32_t *>(&two);
-                        }
-                        dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                } else {
-                    float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((size_t)cp.slot * p.rows + r) * kDv +
-                                                             256 * half + 32 * c);
-#pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4)
-                        dst[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
-                                              __uint_as_float(v[4 * q4 + 2]) * inv,
-                                              __uint_as_float(v[4 * q4 + 3]) * inv);
-                }
-            }
-            if (row_ok && half == 0) {
-                if (whole)
-                    p.lse[((size_t)cp.seq * p.h_q + h_idx) * p.s_q + t_q] = lse;
-                else
-                    p.lse_part[(size_t)cp.slot * p.rows + r] = lse;
-            }
+            tmem_st16(tmem + kTmemPhi + c.lane_off + 16 * c.th, pk);
+            tmem_st16(tmem + kTmemPlo + c.lane_off + 16 * c.th, pl);
+            tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.o_free);
-        ++piece_k;
+        if (c.lane == 0) mbar_arrive(&sm.p_full);
+
+        if (wa.last()) {  // epilogue of this piece: the two token halves' sums, then this warp's O columns
+            sm.xsum[c.th][c.i] = l;
+            named_bar_sync(1, 256);
+            const float l_row = l + sm.xsum[c.th ^ 1][c.i];
+            if (!mbar_wait(&sm.o_full, wa.piece_k & 1, abort)) return;
+            tc_fence_after();
+            if (c.warp_ok) {
+                const Piece &cp = wa.pc;
+                const bool empty = !(l_row > 0.f);
+                const float inv = empty ? 0.f : 1.f / l_row;
+                const bool whole = cp.nsplit == 1;
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t v[32];
+                    const int col = 128 * c.th + 32 * q;
+                    tmem_ld32(tmem + kTmemO + c.lane_off + col, v);
+                    tmem_wait_ld();
+                    if (!c.row_ok) continue;
+                    if (whole) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)cp.seq * p.rows + c.r) * kDv +
+                                                               256 * half + col);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                __nv_bfloat162 two =
+                                    __floats2bfloat162_rn(__uint_as_float(v[8 * q4 + 2 * j]) * inv,
+                                                          __uint_as_float(v[8 * q4 + 2 * j + 1]) * inv);
+                                w[j] = *reinterpret_cast<uint32_t *>(&two);
+                            }
+                            dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    } else {
+                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((size_t)cp.slot * p.rows + c.r) * kDv +
+                                                                 256 * half + col);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
+                                                  __uint_as_float(v[4 * q4 + 2]) * inv,
+                                                  __uint_as_float(v[4 * q4 + 3]) * inv);
+                    }
+                }
+                if (c.row_ok && half == 0 && c.th == 0) {
+                    const float lse = empty ? -INFINITY : (m_ref + log2f(l_row)) * 0.69314718055994530942f;
+                    if (whole)
+                        p.lse[((size_t)cp.seq * p.h_q + h_idx) * p.s_q + t_q] = lse;
+                    else
+                        p.lse_part[(size_t)cp.slot * p.rows + c.r] = lse;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (c.lane == 0) mbar_arrive(&sm.o_free);
+        }
+        // scores of block g+1 (frees the accumulators for Gemm1 of block g+2)
+        if (wb.live) {
+            if (wb.first()) vis = c.row_ok ? visible_keys(wb.pc.n, p.s_q, t_q, p.causal) : 0;
+            if (!load_and_send(sm, c, g + 1, wb.blk * kBlk, vis, e_own, m_own)) return;
+            if (wb.last()) {
+                Cursor tmp = wb.cur;
+                Piece nx;
+                if (tmp.next(p, nx)) load_q(sm, c, nx);
+            }
+        }
+        wa = wb;
     }
 }
 
@@ -452,18 +581,19 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t *meta = p.tile_meta + (size_t)part * kMetaInts;
 
+    if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);  // whole (converged) warp
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.s_free, 4);
-        mbar_init(&sm.p_full, 4);
+        mbar_init(&sm.s_free, 8);
+        mbar_init(&sm.p_full, 8);
         mbar_init(&sm.p_free, 1);
         mbar_init(&sm.o_full, 1);
-        mbar_init(&sm.o_free, 4);
-        mbar_init(&sm.q_full, 4);
+        mbar_init(&sm.o_free, 8);
+        mbar_init(&sm.q_full, 8);
         mbar_init(&sm.mma_done, 1);
         mbar_init(&sm.xfull[0], 1);
         mbar_init(&sm.xfull[1], 1);
@@ -474,7 +604,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
         prefetch_tensormap(&map_lat);
         prefetch_tensormap(&map_rope);
     }
-    if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -494,6 +623,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     if (threadIdx.x == 0 && sm.abort) raise_error(kErrTimeout);
     cluster_sync();  // the peer no longer writes into this CTA's shared memory
     if (warp == 1) {
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
