@@ -215,7 +215,7 @@ __device__ void mma_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, u
     w2 = w1;
     int g1 = 0, g2 = 0;
 
-    // Gemm1 of block g1 into S_a / S_b (two interleaved accumulation chains)
+    // Gemm1 of block g1 into S (partial scores over this CTA's 288 dims)
     auto gemm1 = [&]() -> bool {
         if (w1.first() && !warp_wait(&sm.q_full, w1.piece_k & 1, abort, lane)) return false;
         const int s = g1 % kStages;
@@ -322,7 +322,7 @@ __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &
     if (c.lane == 0) mbar_arrive(&sm.q_full);
 }
 
-// Own partial scores of block g for this thread's 32 tokens: S_a + S_b (log2 units), then
+// Own partial scores of block g for this thread's 32 tokens (log2 units), then
 // E = 2^(s - m) with m the thread's own max; frees the accumulators and sends E (fp16) and m
 // (fp32) to the peer CTA's receive slot g % 2.
 __device__ __forceinline__ bool load_and_send(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&e)[32],
