@@ -178,6 +178,31 @@ int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_b
                     const mla_device_buffers *dev, void *stream);
 
 /*
+ * Decode for callers that cannot allocate device memory (no counterpart on the pages: this
+ * is a library convenience). Same arguments, rules and results as mla_decode, without the
+ * workspace: the fp32 partials of split sequences go to a fixed scratch array of
+ * MLA_NOALLOC_SCRATCH_BYTES that is part of the library's device image (every GPU that
+ * loads the library holds it until the process exits). For callers whose memory comes from
+ * a fixed pool, or whose serving path may not call cudaMalloc (a late allocation can fail
+ * or synchronise), this call allocates nothing: no cudaMalloc, cudaFree or allocating
+ * library routine.
+ *   - Returns MLA_ERR_WORKSPACE, launching nothing, when mla_workspace_bytes(batch, s_q, h_q,
+ *     num_parts) exceeds MLA_NOALLOC_SCRATCH_BYTES (reduce num_parts or the batch).
+ *   - The first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the last call's
+ *     contents (none of which must start at zero): calls that overlap on the GPU, e.g. on
+ *     two streams, race on it and must be serialised by the caller.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int mla_decode_noalloc(const void *q, const void *kv_cache, int64_t num_blocks,
+                       const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                       const int32_t *tile_meta, const int32_t *num_splits, int num_parts,
+                       int batch, int s_q, int h_q, float scale, int causal, void *out, float *lse,
+                       void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's error word.
  * Returns MLA_OK, MLA_ERR_BOUNDS, MLA_ERR_TIMEOUT, or MLA_ERR_CUDA if a CUDA call
  * (including an earlier asynchronous launch) failed.

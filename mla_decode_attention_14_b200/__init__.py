@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # exported C symbols, in the order include/mla.h declares them
 EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
            "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_host",
-           "mla_check_status", "mla_launch_count")
+           "mla_decode_noalloc", "mla_check_status", "mla_launch_count")
 
 
 class MLAError(RuntimeError):
@@ -78,6 +78,8 @@ def lib():
         for name in ("mla_decode", "mla_decode_split"):
             getattr(L, name).argtypes = dec
             getattr(L, name).restype = I
+        L.mla_decode_noalloc.argtypes = dec[:16] + [P]
+        L.mla_decode_noalloc.restype = I
         L.mla_decode_combine.argtypes = [P, I, I, I, I, P, P, P, SZ, P]
         L.mla_decode_combine.restype = I
         L.mla_decode_host.argtypes = [P, P, I64, P, I64, P, I, I, I, F, I, P, P,
@@ -214,6 +216,29 @@ def decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, s
                                                               workspace.data_ptr(), ws_bytes, st))
         else:
             raise ValueError(phase)
+    return out, lse
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20  # MLA_NOALLOC_SCRATCH_BYTES in include/mla.h
+
+
+def decode_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+                   scale: float, causal: bool, meta: Metadata, out: torch.Tensor, lse: torch.Tensor, stream=None):
+    """Decode through ``mla_decode_noalloc``: no workspace, no device allocation by the library.
+
+    For callers that cannot allocate device memory at decode time (fixed memory pools, serving
+    paths where a late allocation could fail or stall): the split partials go to the library's
+    fixed scratch array (``NOALLOC_SCRATCH_BYTES``), shared by every call on the device, so calls
+    must not overlap on the GPU. ``out`` and ``lse`` are caller-provided.
+    """
+    b, s_q, h_q = _decode_args(q, kv_cache, block_table, seqlens, meta)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    with torch.cuda.device(q.device):
+        _check("mla_decode_noalloc", lib().mla_decode_noalloc(
+            q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(), block_table.shape[1],
+            seqlens.data_ptr(), meta.tile_meta.data_ptr(), meta.num_splits.data_ptr(), meta.num_parts, b, s_q, h_q,
+            float(scale), int(bool(causal)), out.data_ptr(), lse.data_ptr(), _stream(stream)))
     return out, lse
 
 

@@ -4,3 +4,4 @@
 #include "metadata.cu"
 #include "combine.cu"
 #include "decode_sm100.cu"
+#include "noalloc.cu"

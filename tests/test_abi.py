@@ -98,3 +98,21 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         mla.get_metadata(torch.zeros(4, dtype=torch.int32), 16, 1, num_parts=4, fixed_cost=5)
+
+
+def test_noalloc_rejects_oversized_requests_on_host(L):
+    # beyond MLA_NOALLOC_SCRATCH_BYTES: rejected before any CUDA call (this host has no GPU)
+    big_parts = 60000
+    assert L.mla_workspace_bytes(2, 1, 128, big_parts) > mla.NOALLOC_SCRATCH_BYTES
+    rc = L.mla_decode_noalloc(FAKE, FAKE, 10, FAKE, 4, FAKE, FAKE, FAKE, big_parts, 2, 1, 128, 0.1, 0,
+                              FAKE, FAKE, None)
+    assert rc == 3  # MLA_ERR_WORKSPACE
+    assert L.mla_decode_noalloc(None, FAKE, 10, FAKE, 4, FAKE, FAKE, FAKE, 4, 2, 1, 16, 0.1, 0,
+                                FAKE, FAKE, None) == 1  # MLA_ERR_INVALID_ARG
+
+
+def test_noalloc_scratch_constant_matches_header():
+    import re
+    src = open(HEADER).read()
+    m = re.search(r"#define MLA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", src)
+    assert m and int(m.group(1)) << int(m.group(2)) == mla.NOALLOC_SCRATCH_BYTES
