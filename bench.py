@@ -135,6 +135,24 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, device=None):
+    """Elementwise max of per-rank timings over all ranks (identity without a process group).
+
+    Every rank must call this the same number of times, in the same order."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job TB/s: every rank decodes its own batch of the same shape (weak scaling)."""
+    return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, wl, inp, counts):
     import oracle
@@ -304,15 +322,10 @@ def main():
     if st != 0:
         raise SystemExit("device error status %d in the timed region" % st)
 
-    if dist is not None:
-        t = torch.tensor([total_ms, statistics.mean(split_ms)], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, split_avg_ms = float(t[0]), float(t[1])
-    else:
-        split_avg_ms = statistics.mean(split_ms)
+    total_ms, split_avg_ms = max_over_ranks([total_ms, statistics.mean(split_ms)], dev)
     ms_per_step = total_ms / args.steps
     bytes_all = counts["bytes"] * world
-    value = bytes_all / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(counts["bytes"], world, ms_per_step)
     tflops = counts["flops"] * world / (ms_per_step * 1e-3) / 1e12
 
     # end to end through the host entry point: pinned host inputs in, host outputs out
@@ -337,11 +350,7 @@ def main():
             hd(qh, kvh, bth, slh, wl.scale, wl.causal, oh, lh)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dev)[0]
         h2d = sum(x.numel() * x.element_size() for x in (qh, kvh, bth, slh))
         d2h = oh.numel() * 2 + lh.numel() * 4
         e2e = {"value": bytes_all / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
