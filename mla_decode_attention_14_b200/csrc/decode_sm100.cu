@@ -15,31 +15,35 @@
 //    [256h, 256h+256) and rotary dims [512+32h, 512+32h+32), i.e. exactly half of every block
 //    (36,864 bytes); the pair together reads each block once.
 //  * Gemm1 is split along its 576-long contraction: CTA h computes the partial scores over its
-//    288 dims (18 tcgen05 MMAs, M=128 rows, N=64 tokens; the latent part of Q is the A operand
+//    288 dims (18 tcgen05 MMAs, M=128 rows, N=64 tokens, into two accumulators of 9 k-steps each
+//    so that consecutive MMAs do not wait on one another; the latent part of Q is the A operand
 //    in TMEM, the rotary part in shared memory).
 //  * The pair combines the partial scores multiplicatively: 2^(s0 + s1 - m) =
-//    2^(s0 - m0) * 2^(s1 - m1) * 2^(m0 + m1 - m). Each CTA computes E = 2^(s - m) for its own
-//    partial with its own row offset m, keeps it in fp32, and sends it to the peer as fp16
-//    (scaled by 2^15) together with m in fp32: st.async stores into the peer's 2-slot receive
-//    ring complete on the peer's mbarrier. The relative error of the exchanged factor is that
-//    of fp16 (2^-11) whatever the score magnitude, and the traffic is half that of fp32 scores.
+//    2^(s0 - m0) * 2^(s1 - m1) * 2^(m0 + m1 - m). Each CTA computes E = 2^(s - m + 15) for its
+//    own partial with its own row offset m, keeps it in fp32, and sends it to the peer as fp16
+//    together with m in fp32: st.async stores into the peer's 2-slot receive ring complete on
+//    the peer's mbarrier. E lies in (0, 2^15], so the exchanged factor keeps fp16's relative
+//    precision (2^-11) down to 2^-29 of the row max whatever the score magnitude, and the
+//    traffic is half that of fp32 scores.
 //  * Eight softmax warps: warp w serves TMEM lane quarter w&3 (32 query rows) and one half of
 //    every block's tokens; the two halves of a row agree on an upper bound of the block max
 //    through shared memory, so both take the same lazy-rescaling decisions (O is rescaled only
-//    when the running max grows by more than 2^8). P = E_own * E_peer * 2^(m0 + m1 - m) goes
-//    to TMEM as two bf16 terms, hi = bf16(P) and lo = bf16(P - hi), so P's rounding does not
-//    add to the bf16 output rounding.
+//    when the running max grows by more than 2^8). P = E_own * E_peer * 2^(m0 + m1 - m - 30) goes
+//    to shared memory as two bf16 terms (hi = P with its low 16 bits cleared, lo = the exact
+//    remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P), so P's rounding
+//    does not add to the bf16 output rounding.
 //  * Issuing a tcgen05 MMA blocks the issuing thread until the tensor core takes it, so the MMA
 //    warp's program order is the tensor-core schedule: Gemm1 of block g+1 runs while the softmax
 //    warps finish block g, Gemm2 of block g right after.
-//  * Gemm2: 8 MMAs (M=128, N=256, K=16 tokens; A = P_hi then P_lo from TMEM, B = the value half
-//    of the same shared-memory tile read MN-major): the block is loaded once for both GEMMs.
+//  * Gemm2: 8 MMAs (M=128, N=256, K=16 tokens; A = P_hi then P_lo, K-major in shared memory,
+//    B = the value half of the same cache tile read MN-major): the block is loaded once for
+//    both GEMMs.
 //  * Warp roles: warp 0 lane 0 = TMA producer (4-stage ring, block-table gather, L2
 //    evict-first); warp 1 = MMA warp (lane 0 issues; the warp owns the TMEM allocation and
 //    zeroes the cache rows past a sequence's end before any MMA reads them, so undefined
 //    tail contents never reach the result); warps 4-11 = softmax, correction and epilogue
-//    (warps 2-3 idle: the softmax warps must start at a multiple of 4 so that warp w serves
-//    TMEM lane quarter w & 3).
+//    (a warp may only touch TMEM lane quarter w & 3; warps 2-3 idle, so that warpgroup 0 can
+//    hand its registers to the two softmax warpgroups).
 //  * Pieces of split sequences leave fp32 partial O and lse in the workspace for the combine
 //    kernel; whole sequences are written straight to bf16 out / fp32 lse.
 // Every wait is bounded; a timeout sets the device error word and the CTA exits cleanly.
@@ -54,25 +58,30 @@ using namespace sm100;
 namespace dec {
 constexpr int kStages = 4;
 constexpr int kThreads = 384;
+constexpr int kFirstSoftWarp = 4;
+// Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 = 64,512); warpgroup 0
+// (producer, MMA, two idle warps) drops to 96 and the two softmax warpgroups rise to 200:
+// 128 x 96 + 256 x 200 = 63,488 <= 64,512.
+constexpr uint32_t kRegsControl = 96, kRegsSoftmax = 200;
 constexpr int kBoxBytes = kBlk * 128;                      // 64 tokens x 64 bf16 (128-byte swizzle)
 constexpr int kRopeBoxBytes = kBlk * 64;                   // 64 tokens x 32 bf16 (64-byte swizzle)
 constexpr int kStageBytes = 4 * kBoxBytes + kRopeBoxBytes;  // 36,864: half of one cache block
 constexpr float kRescaleThreshold = 8.0f;                  // log2 units: rescale O when max grows > 2^8
-// The peer's factors E = 2^(s - m) <= 1 cross the cluster as fp16 scaled by 2^15 (< 65504), which
-// keeps values down to 2^-29 normal (full 11-bit precision); the receiver folds 2^-15 back in.
-constexpr float kXScale = 32768.0f;
+// The factors E = 2^(s - m + 15) <= 2^15 (< 65504) cross the cluster as fp16, normal (full 11-bit
+// precision) down to 2^-29 of the row max; P folds the two 2^15 back out.
 constexpr float kXScaleLog2 = 15.0f;
 
 // TMEM column map (512 columns allocated, 128 lanes = 128 query rows)
 constexpr uint32_t kTmemO = 0;     // 256 fp32: O for this CTA's 256 value dims
 constexpr uint32_t kTmemQ = 256;   // 128 x (2 bf16): this CTA's 256 latent query dims
-constexpr uint32_t kTmemS = 384;   // 64 fp32: partial scores of the current block
-constexpr uint32_t kTmemPhi = 448; // 32 x (2 bf16): P rounded to bf16
-constexpr uint32_t kTmemPlo = 480; // 32 x (2 bf16): bf16 of P's rounding residue
+constexpr uint32_t kTmemSa = 384;  // 64 fp32: partial scores, first half of the k-steps
+constexpr uint32_t kTmemSb = 448;  // 64 fp32: partial scores, second half of the k-steps
 constexpr uint32_t kTmemCols = 512;
+constexpr int kPTileBytes = 128 * 128;  // 128 rows x 64 tokens bf16, K-major, 128-byte swizzle
 
 struct __align__(1024) Smem {
     uint8_t stage[kStages][kStageBytes];  // KV ring
+    uint8_t p_tile[2][kPTileBytes];       // P of the current block: [0] = bf16 high part, [1] = low part
     uint4 xchg[2 * 2 * 4 * 128 + 2 * 2 * 128 / 4];  // peer E factors (fp16) [slot][token half][16 B][row]
                                                     // + row offsets (fp32) [slot][token half][row]
     float xmax[2][2][128], xsum[2][128];            // per-row exchange between the two token halves
@@ -228,13 +237,18 @@ __device__ void mma_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, u
             const uint64_t kd = smem_desc(smem_addr(sm.stage[s]), 16, 1024, 2);
             const uint64_t rd = smem_desc(smem_addr(sm.stage[s]) + 4 * kBoxBytes, 16, 512, 4);
             const uint64_t qd = smem_desc(smem_addr(sm.q_rope), 16, 512, 4);
+            // two independent accumulators (k-steps 0-7 + rotary 0, k-steps 8-15 + rotary 1): a chain of
+            // dependent MMAs into one accumulator runs at about half the tensor core's rate
 #pragma unroll
-            for (int k = 0; k < 16; ++k)  // latent k-steps, A (Q) from TMEM
-                mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * k,
+            for (int k = 0; k < 8; ++k) {  // latent k-steps, A (Q) from TMEM
+                mma_ts(tmem + kTmemSa, tmem + kTmemQ + 8 * k,
                        kd + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id1, k > 0 ? 1u : 0u);
+                mma_ts(tmem + kTmemSb, tmem + kTmemQ + 8 * (k + 8),
+                       kd + (uint64_t)((((k + 8) >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id1, k > 0 ? 1u : 0u);
+            }
 #pragma unroll
             for (int c = 0; c < 2; ++c)  // rotary k-steps, A from shared memory
-                mma_ss(tmem + kTmemS, qd + 2 * c, rd + 2 * c, id1, 1u);
+                mma_ss(tmem + (c ? kTmemSb : kTmemSa), qd + 2 * c, rd + 2 * c, id1, 1u);
             mma_commit(&sm.s_full);
         }
         __syncwarp();
@@ -252,12 +266,13 @@ __device__ void mma_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, u
         if (lane == 0) {
             tc_fence_after();
             const uint64_t vd = smem_desc(smem_addr(sm.stage[g2 % kStages]), 4 * 2048, 1024, 2);
+            const uint64_t pd = smem_desc(smem_addr(sm.p_tile[0]), 16, 1024, 2);
             const bool first = w2.first();
 #pragma unroll
-            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo: O += (P_hi + P_lo) V, A from TMEM
+            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo: O += (P_hi + P_lo) V, both from shared memory
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + kTmemO, tmem + (hl ? kTmemPlo : kTmemPhi) + 8 * kk, vd + 128 * kk, id2,
+                    mma_ss(tmem + kTmemO, pd + (uint64_t)((hl * kPTileBytes + 32 * kk) >> 4), vd + 128 * kk, id2,
                            (!first || hl > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&sm.p_free);
             mma_commit(&sm.kv_empty[g2 % kStages]);
@@ -322,24 +337,31 @@ __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &
     if (c.lane == 0) mbar_arrive(&sm.q_full);
 }
 
-// Own partial scores of block g for this thread's 32 tokens (log2 units), then
-// E = 2^(s - m) with m the thread's own max; frees the accumulators and sends E (fp16) and m
-// (fp32) to the peer CTA's receive slot g % 2.
+// Own partial scores of block g for this thread's 32 tokens. The accumulators are released as
+// soon as they are in registers; then E = 2^(s - m + 15) with m the thread's own max (log2
+// units), and E (fp16) and m (fp32) go to the peer CTA's receive slot g % 2. E stays in fp32
+// here, in (0, 2^15].
 __device__ __forceinline__ bool load_and_send(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&e)[32],
                                               float &m_own) {
     if (!mbar_wait(&sm.s_full, g & 1, &sm.abort)) return false;
     tc_fence_after();
+    if (c.warp_ok) {
+        uint32_t a[32], b[32];
+        tmem_ld32(c.tmem + kTmemSa + c.lane_off + 32 * c.th, a);
+        tmem_ld32(c.tmem + kTmemSb + c.lane_off + 32 * c.th, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) e[j] = __uint_as_float(a[j]) + __uint_as_float(b[j]);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&sm.s_free);
     m_own = -INFINITY;
     if (c.warp_ok) {
-        uint32_t a[32];
-        tmem_ld32(c.tmem + kTmemS + c.lane_off + 32 * c.th, a);
-        tmem_wait_ld();
-        const float sl2 = c.p->scale_log2;
         const int k0 = key0 + 32 * c.th;
+        if (k0 + 32 > vis) {  // the sequence ends (or the causal limit falls) inside these tokens
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const float v = __uint_as_float(a[j]) * sl2;
-            e[j] = k0 + j < vis ? v : -INFINITY;
+            for (int j = 0; j < 32; ++j) e[j] = k0 + j < vis ? e[j] : -INFINITY;
         }
         float t[16];
 #pragma unroll
@@ -348,15 +370,12 @@ __device__ __forceinline__ bool load_and_send(Smem &sm, const SoftCtx &c, int g,
         for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
             for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
-        m_own = t[0];
-        const bool none = m_own == -INFINITY;
+        const float sl2 = c.p->scale_log2;  // > 0, so the max commutes with the scaling
+        const bool none = t[0] == -INFINITY;
+        m_own = none ? -INFINITY : t[0] * sl2;
+        const float off = none ? 0.f : kXScaleLog2 - m_own;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) e[j] = none ? 0.f : ex2_approx(e[j] - m_own);
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (c.lane == 0) mbar_arrive(&sm.s_free);
-    if (c.warp_ok) {
+        for (int j = 0; j < 32; ++j) e[j] = none ? 0.f : ex2_approx(fmaf(e[j], sl2, off));
         const int slot = g & 1;
         const uint32_t base = c.xchg_peer + (uint32_t)(((slot * 2 + c.th) * 4) * 128 + c.i) * 16;
         const uint32_t bar = c.xfull_peer0 + slot * 8;
@@ -365,14 +384,14 @@ __device__ __forceinline__ bool load_and_send(Smem &sm, const SoftCtx &c, int g,
             uint32_t w[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                __half2 two = __floats2half2_rn(e[8 * c4 + 2 * q] * kXScale, e[8 * c4 + 2 * q + 1] * kXScale);
+                __half2 two = __floats2half2_rn(e[8 * c4 + 2 * q], e[8 * c4 + 2 * q + 1]);
                 w[q] = *reinterpret_cast<uint32_t *>(&two);
             }
             st_async_v4_b32(base + c4 * 128 * 16, w[0], w[1], w[2], w[3], bar);
         }
         // the row offset travels in the offsets area of the same slot
-        const uint32_t off = c.xchg_peer + (uint32_t)(2 * 2 * 4 * 128 * 16) + (uint32_t)((slot * 2 + c.th) * 128 + c.i) * 4;
-        st_async_b32(off, __float_as_uint(m_own), bar);
+        const uint32_t offa = c.xchg_peer + (uint32_t)(2 * 2 * 4 * 128 * 16) + (uint32_t)((slot * 2 + c.th) * 128 + c.i) * 4;
+        st_async_b32(offa, __float_as_uint(m_own), bar);
     }
     return true;
 }
@@ -385,7 +404,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     c.half = half;
     const int warp = threadIdx.x >> 5;
     const int wq = warp & 3;
-    c.th = (warp - 4) >> 2;
+    c.th = (warp - kFirstSoftWarp) >> 2;
     c.lane = threadIdx.x & 31;
     c.i = wq * 32 + c.lane;  // row within the group == TMEM lane
     c.lane_off = (uint32_t)(wq * 32) << 16;
@@ -420,7 +439,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         wb.advance(p);
         // peer factors of block g (slot g % 2)
         const int slot = g & 1;
-        if (threadIdx.x == 128) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
+        if (threadIdx.x == 32 * kFirstSoftWarp) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
         if (!mbar_wait_cluster(&sm.xfull[slot], (g >> 1) & 1, abort)) return;
         float e_peer[32];
         float m_peer = -INFINITY;
@@ -442,7 +461,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         // an upper bound of the block's row max (both token halves), shared by the two warps of a row
         const float mbu_half = m_own + m_peer;
         sm.xmax[g & 1][c.th][c.i] = mbu_half;
-        named_bar_sync(1, 256);
+        named_bar_sync(1 + (c.i >> 5), 64);  // the two warps of these 32 rows
         const float mbu = fmaxf(mbu_half, sm.xmax[g & 1][c.th ^ 1][c.i]);
         bool need = false;
         float alpha = 1.f;
@@ -459,22 +478,26 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 need = true;
             }
         }
-        uint32_t pk[16], pl[16];  // P rounded to bf16 (hi) and the bf16 of its rounding residue (lo)
+        // P = 2^(s0 + s1 - m_ref) in two bf16 terms: hi = P with its low 16 bits cleared, lo = the
+        // (exact) remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P.
+        uint32_t pk[16], pl[16];
         if (c.warp_ok) {
             const bool none = m_ref == -INFINITY || mbu_half == -INFINITY;
-            const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - kXScaleLog2);
+            const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 2.f * kXScaleLog2);
             float su[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
                 const float p0 = e_own[j] * e_peer[j] * f, p1 = e_own[j + 1] * e_peer[j + 1] * f;
                 su[(j >> 1) & 3] += p0 + p1;
-                const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-                const float2 hf = __bfloat1622float2(hi);
-                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-                pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&hi);
-                pl[j >> 1] = *reinterpret_cast<const uint32_t *>(&lo);
+                const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
+                pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
             }
             l += (su[0] + su[1]) + (su[2] + su[3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = pl[j] = 0u;
         }
         // the P tile and O are free once Gemm2 of block g-1 has completed
         if (g > 0 && !mbar_wait(&sm.p_free, (g - 1) & 1, abort)) return;
@@ -493,9 +516,16 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 }
                 tmem_wait_st();
             }
-            tmem_st16(tmem + kTmemPhi + c.lane_off + 16 * c.th, pk);
-            tmem_st16(tmem + kTmemPlo + c.lane_off + 16 * c.th, pl);
-            tmem_wait_st();
+        }
+        {  // this thread's 64 bytes of row i in both P tiles (K-major, 128-byte swizzle)
+            uint8_t *row_hi = sm.p_tile[0] + c.i * 128, *row_lo = sm.p_tile[1] + c.i * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int chunk = ((4 * c.th + q) ^ (c.i & 7)) * 16;
+                *reinterpret_cast<uint4 *>(row_hi + chunk) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                *reinterpret_cast<uint4 *>(row_lo + chunk) = make_uint4(pl[4 * q], pl[4 * q + 1], pl[4 * q + 2], pl[4 * q + 3]);
+            }
+            fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
         }
         tc_fence_before();
         __syncwarp();
@@ -503,7 +533,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
 
         if (wa.last()) {  // epilogue of this piece: the two token halves' sums, then this warp's O columns
             sm.xsum[c.th][c.i] = l;
-            named_bar_sync(1, 256);
+            named_bar_sync(1 + (c.i >> 5), 64);
             const float l_row = l + sm.xsum[c.th ^ 1][c.i];
             if (!mbar_wait(&sm.o_full, wa.piece_k & 1, abort)) return;
             tc_fence_after();
@@ -610,11 +640,15 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     cluster_sync();  // the peer's barriers exist before any exchange targets them
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0) {
-        if (lane == 0) producer(sm, p, &map_lat, &map_rope, meta, half);
-    } else if (warp == 1) {
-        mma_warp(sm, p, meta, tmem);
-    } else if (warp >= 4) {
+    if (warp < kFirstSoftWarp) {
+        setmaxnreg_dec<kRegsControl>();
+        if (warp == 0) {
+            if (lane == 0) producer(sm, p, &map_lat, &map_rope, meta, half);
+        } else if (warp == 1) {
+            mma_warp(sm, p, meta, tmem);
+        }
+    } else {
+        setmaxnreg_inc<kRegsSoftmax>();
         softmax_role(sm, p, meta, tmem, half, group);
     }
     __syncwarp();

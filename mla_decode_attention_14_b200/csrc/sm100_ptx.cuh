@@ -188,6 +188,16 @@ MLA_DEV void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
                  : "memory");
 }
 MLA_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Per-warpgroup register budget (every warp of the warpgroup executes the same call).
+template <uint32_t N>
+MLA_DEV void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <uint32_t N>
+MLA_DEV void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 MLA_DEV void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
