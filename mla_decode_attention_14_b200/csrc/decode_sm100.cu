@@ -32,18 +32,17 @@
 //    to shared memory as two bf16 terms (hi = P with its low 16 bits cleared, lo = the exact
 //    remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P), so P's rounding
 //    does not add to the bf16 output rounding.
-//  * Issuing a tcgen05 MMA blocks the issuing thread until the tensor core takes it, so the MMA
-//    warp's program order is the tensor-core schedule: Gemm1 of block g+1 runs while the softmax
-//    warps finish block g, Gemm2 of block g right after.
+//  * Issuing a tcgen05 MMA occupies the issuing thread for about 70 cycles, so three warps issue:
+//    one per Gemm1 accumulator and one for Gemm2. The softmax warps read the scores of block g+1
+//    before they finish block g, so Gemm1 of block g+2 can start while Gemm2 of block g waits for P.
 //  * Gemm2: 8 MMAs (M=128, N=256, K=16 tokens; A = P_hi then P_lo, K-major in shared memory,
 //    B = the value half of the same cache tile read MN-major): the block is loaded once for
 //    both GEMMs.
 //  * Warp roles: warp 0 lane 0 = TMA producer (4-stage ring, block-table gather, L2
-//    evict-first); warp 1 = MMA warp (lane 0 issues; the warp owns the TMEM allocation and
-//    zeroes the cache rows past a sequence's end before any MMA reads them, so undefined
-//    tail contents never reach the result); warps 4-11 = softmax, correction and epilogue
-//    (a warp may only touch TMEM lane quarter w & 3; warps 2-3 idle, so that warpgroup 0 can
-//    hand its registers to the two softmax warpgroups).
+//    evict-first); warps 1-2 issue Gemm1 (warp 1 also owns the TMEM allocation); warp 3 issues
+//    Gemm2 and zeroes the cache rows past a sequence's end before Gemm2 reads them, so undefined
+//    tail contents never reach the result; warps 4-11 = softmax, correction and epilogue (a warp
+//    may only touch TMEM lane quarter w & 3). Warpgroup 0 hands registers to the softmax warps.
 //  * Pieces of split sequences leave fp32 partial O and lse in the workspace for the combine
 //    kernel; whole sequences are written straight to bf16 out / fp32 lse.
 // Every wait is bounded; a timeout sets the device error word and the CTA exits cleanly.
@@ -57,11 +56,13 @@ using namespace sm100;
 
 namespace dec {
 constexpr int kStages = 4;
-constexpr int kThreads = 384;
-constexpr int kFirstSoftWarp = 4;
+constexpr int kFirstSoftWarp = 4;                 // warpgroup 0: TMA producer and the three MMA-issuing warps
+constexpr int kSoftWarps = 8;                     // two per SM sub-partition
+constexpr int kThreads = 32 * (kFirstSoftWarp + kSoftWarps);  // 384
+constexpr int kTq = 2;                            // token halves per block
+constexpr int kTokPer = kBlk / kTq;               // 32 tokens per softmax thread
 // Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 = 64,512); warpgroup 0
-// (producer, MMA, two idle warps) drops to 96 and the two softmax warpgroups rise to 200:
-// 128 x 96 + 256 x 200 = 63,488 <= 64,512.
+// drops to 96 and the two softmax warpgroups rise to 200: 128 x 96 + 256 x 200 = 63,488 <= 64,512.
 constexpr uint32_t kRegsControl = 96, kRegsSoftmax = 200;
 constexpr int kBoxBytes = kBlk * 128;                      // 64 tokens x 64 bf16 (128-byte swizzle)
 constexpr int kRopeBoxBytes = kBlk * 64;                   // 64 tokens x 32 bf16 (64-byte swizzle)
@@ -78,13 +79,15 @@ constexpr uint32_t kTmemSa = 384;  // 64 fp32: partial scores, first half of the
 constexpr uint32_t kTmemSb = 448;  // 64 fp32: partial scores, second half of the k-steps
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPTileBytes = 128 * 128;  // 128 rows x 64 tokens bf16, K-major, 128-byte swizzle
+constexpr int kXchgEBytes = 2 * kBlk * 128 * 2;    // two slots of 128 rows x 64 fp16 factors
+constexpr int kXchgOffBytes = 2 * kTq * 128 * 4;   // two slots of 128 rows x 2 fp32 offsets
 
 struct __align__(1024) Smem {
     uint8_t stage[kStages][kStageBytes];  // KV ring
     uint8_t p_tile[2][kPTileBytes];       // P of the current block: [0] = bf16 high part, [1] = low part
-    uint4 xchg[2 * 2 * 4 * 128 + 2 * 2 * 128 / 4];  // peer E factors (fp16) [slot][token half][16 B][row]
-                                                    // + row offsets (fp32) [slot][token half][row]
-    float xmax[2][2][128], xsum[2][128];            // per-row exchange between the two token halves
+    uint4 xchg[(kXchgEBytes + kXchgOffBytes) / 16];  // peer E factors (fp16) [slot][token half][16 B][row]
+                                                     // + row offsets (fp32) [slot][token half][row]
+    float xmax[2][kTq][128];  // per-row exchange between the two token halves (block max bound; sums)
     uint8_t q_rope[128 * 64];             // rotary query dims [128 rows x 32], K-major, 64-byte swizzle
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full, s_free, p_full, p_free, o_full, o_free, q_full, mma_done;
@@ -187,12 +190,12 @@ __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map
     // every load still in flight must land before the CTA may exit
     for (int k = max(0, gidx - kStages); k < gidx; ++k) {
         const long long t0 = clock64();
-        while (!mbar_test(&sm.kv_full[k % kStages], (k / kStages) & 1) && clock64() - t0 < kSpinCycles) {
+        while (!mbar_sleep_test(&sm.kv_full[k % kStages], (k / kStages) & 1) && clock64() - t0 < kSpinCycles) {
         }
     }
 }
 
-// ---------------------------------------------------------------- MMA warp
+// ---------------------------------------------------------------- MMA issuing warps
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int lane) {
     bool ok = true;
     if (lane == 0) ok = mbar_wait(bar, parity, abort);
@@ -214,80 +217,81 @@ __device__ void zero_tail_rows(uint8_t *st, int valid, int lane) {
     __syncwarp();
 }
 
-__device__ void mma_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
-    constexpr uint32_t id1 = idesc_bf16_f32(128, 64, 0);   // S = Q K^T: K-major B
-    constexpr uint32_t id2 = idesc_bf16_f32(128, 256, 1);  // O += P V: MN-major B
+// Issuing one tcgen05 MMA occupies the issuing thread for about 70 cycles whatever its size, so
+// the small Gemm1 MMAs (N = 64) are spread over two issuing warps, one per accumulator, and
+// Gemm2 has a third: the tensor core takes MMAs from all three at once.
+
+// Gemm1 of every block into accumulator `which` (0: latent k-steps 0-7 + rotary k-step 0 into S_a,
+// 1: latent k-steps 8-15 + rotary k-step 1 into S_b); s_full completes once both have landed.
+__device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem, int which) {
+    constexpr uint32_t id1 = idesc_bf16_f32(128, 64, 0);  // S = Q K^T: K-major B
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
-    BlockWalker w1, w2;  // w1: next Gemm1, w2: next Gemm2 (one block behind)
-    w1.init(meta, p);
-    w2 = w1;
-    int g1 = 0, g2 = 0;
-
-    // Gemm1 of block g1 into S (partial scores over this CTA's 288 dims)
-    auto gemm1 = [&]() -> bool {
-        if (w1.first() && !warp_wait(&sm.q_full, w1.piece_k & 1, abort, lane)) return false;
-        const int s = g1 % kStages;
-        if (!warp_wait(&sm.kv_full[s], (g1 / kStages) & 1, abort, lane)) return false;
-        if (w1.tail()) zero_tail_rows(sm.stage[s], w1.pc.n - w1.blk * kBlk, lane);
-        if (g1 > 0 && !warp_wait(&sm.s_free, (g1 - 1) & 1, abort, lane)) return false;
+    const uint32_t d = tmem + (which ? kTmemSb : kTmemSa);
+    BlockWalker w;
+    w.init(meta, p);
+    for (int g = 0; w.live; w.advance(p), ++g) {
+        if (w.first() && !warp_wait(&sm.q_full, w.piece_k & 1, abort, lane)) break;
+        const int s = g % kStages;
+        if (!warp_wait(&sm.kv_full[s], (g / kStages) & 1, abort, lane)) break;
+        if (g > 0 && !warp_wait(&sm.s_free, (g - 1) & 1, abort, lane)) break;
         if (lane == 0) {
             tc_fence_after();
             // descriptors: one base each, then constant offsets (address field is in 16-byte units)
             const uint64_t kd = smem_desc(smem_addr(sm.stage[s]), 16, 1024, 2);
             const uint64_t rd = smem_desc(smem_addr(sm.stage[s]) + 4 * kBoxBytes, 16, 512, 4);
             const uint64_t qd = smem_desc(smem_addr(sm.q_rope), 16, 512, 4);
-            // two independent accumulators (k-steps 0-7 + rotary 0, k-steps 8-15 + rotary 1): a chain of
-            // dependent MMAs into one accumulator runs at about half the tensor core's rate
 #pragma unroll
             for (int k = 0; k < 8; ++k) {  // latent k-steps, A (Q) from TMEM
-                mma_ts(tmem + kTmemSa, tmem + kTmemQ + 8 * k,
-                       kd + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id1, k > 0 ? 1u : 0u);
-                mma_ts(tmem + kTmemSb, tmem + kTmemQ + 8 * (k + 8),
-                       kd + (uint64_t)((((k + 8) >> 2) * kBoxBytes + (k & 3) * 32) >> 4), id1, k > 0 ? 1u : 0u);
+                const int kk = 8 * which + k;
+                mma_ts(d, tmem + kTmemQ + 8 * kk, kd + (uint64_t)(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4), id1,
+                       k > 0 ? 1u : 0u);
             }
-#pragma unroll
-            for (int c = 0; c < 2; ++c)  // rotary k-steps, A from shared memory
-                mma_ss(tmem + (c ? kTmemSb : kTmemSa), qd + 2 * c, rd + 2 * c, id1, 1u);
+            mma_ss(d, qd + 2 * which, rd + 2 * which, id1, 1u);  // rotary k-step, A from shared memory
             mma_commit(&sm.s_full);
         }
         __syncwarp();
-        ++g1;
-        w1.advance(p);
-        return true;
-    };
+    }
+}
 
-    if (w1.live && !gemm1()) goto done;
-    while (w2.live) {
-        if (w1.live && !gemm1()) goto done;
-        // Gemm2 of block g2: O (+)= P V
-        if (!warp_wait(&sm.p_full, g2 & 1, abort, lane)) goto done;
-        if (w2.first() && w2.piece_k > 0 && !warp_wait(&sm.o_free, (w2.piece_k - 1) & 1, abort, lane)) goto done;
+// Gemm2 of every block, O (+)= (P_hi + P_lo) V, once the softmax warps have written P.
+__device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
+    constexpr uint32_t id2 = idesc_bf16_f32(128, 256, 1);  // MN-major B
+    const int lane = threadIdx.x & 31;
+    volatile int *abort = &sm.abort;
+    BlockWalker w;
+    w.init(meta, p);
+    for (int g = 0; w.live; w.advance(p), ++g) {
+        if (!warp_wait(&sm.p_full, g & 1, abort, lane)) break;
+        if (w.first() && w.piece_k > 0 && !warp_wait(&sm.o_free, (w.piece_k - 1) & 1, abort, lane)) break;
+        const int s = g % kStages;
+        // P of block g exists, so Gemm1 of block g has completed and its tile may be edited
+        if (w.tail()) zero_tail_rows(sm.stage[s], w.pc.n - w.blk * kBlk, lane);
         if (lane == 0) {
             tc_fence_after();
-            const uint64_t vd = smem_desc(smem_addr(sm.stage[g2 % kStages]), 4 * 2048, 1024, 2);
+            const uint64_t vd = smem_desc(smem_addr(sm.stage[s]), 4 * 2048, 1024, 2);
             const uint64_t pd = smem_desc(smem_addr(sm.p_tile[0]), 16, 1024, 2);
-            const bool first = w2.first();
+            const bool first = w.first();
 #pragma unroll
-            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo: O += (P_hi + P_lo) V, both from shared memory
+            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo, both K-major in shared memory
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_ss(tmem + kTmemO, pd + (uint64_t)((hl * kPTileBytes + 32 * kk) >> 4), vd + 128 * kk, id2,
                            (!first || hl > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&sm.p_free);
-            mma_commit(&sm.kv_empty[g2 % kStages]);
-            if (w2.last()) mma_commit(&sm.o_full);
+            mma_commit(&sm.kv_empty[s]);
+            if (w.last()) mma_commit(&sm.o_full);
         }
         __syncwarp();
-        ++g2;
-        w2.advance(p);
     }
-done:
-    // all issued MMAs complete before teardown (bounded; independent of the abort flag)
-    if (lane == 0) {
+}
+
+// Every MMA an issuing warp started completes before teardown (bounded; independent of the abort flag).
+__device__ void drain_mmas(Smem &sm) {
+    if ((threadIdx.x & 31) == 0) {
         mma_commit(&sm.mma_done);
         const long long t0 = clock64();
-        while (!mbar_test(&sm.mma_done, 0) && clock64() - t0 < kSpinCycles) {
+        while (!mbar_sleep_test(&sm.mma_done, 0) && clock64() - t0 < kSpinCycles) {
         }
     }
     __syncwarp();
@@ -305,7 +309,7 @@ struct SoftCtx {
 };
 
 // Q of piece `pc`: latent half -> TMEM (this warp's lanes, its 64 of the 128 columns),
-// rotary half -> shared memory (its 2 of the 4 chunks of the row).
+// rotary half -> shared memory (its 2 of the 4 16-byte chunks of the row).
 __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &pc) {
     if (c.warp_ok) {
         const DecodeParams &p = *c.p;
@@ -337,63 +341,69 @@ __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &
     if (c.lane == 0) mbar_arrive(&sm.q_full);
 }
 
-// Own partial scores of block g for this thread's 32 tokens. The accumulators are released as
-// soon as they are in registers; then E = 2^(s - m + 15) with m the thread's own max (log2
-// units), and E (fp16) and m (fp32) go to the peer CTA's receive slot g % 2. E stays in fp32
-// here, in (0, 2^15].
-__device__ __forceinline__ bool load_and_send(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&e)[32],
-                                              float &m_own) {
+// Own partial scores of block g for this thread's 32 tokens (raw, unscaled); keys at or past `vis`
+// become -inf. The accumulators are released as soon as the scores are in registers.
+__device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&s)[kTokPer]) {
     if (!mbar_wait(&sm.s_full, g & 1, &sm.abort)) return false;
     tc_fence_after();
-    if (c.warp_ok) {
+    {
         uint32_t a[32], b[32];
-        tmem_ld32(c.tmem + kTmemSa + c.lane_off + 32 * c.th, a);
-        tmem_ld32(c.tmem + kTmemSb + c.lane_off + 32 * c.th, b);
+        tmem_ld32(c.tmem + kTmemSa + c.lane_off + kTokPer * c.th, a);
+        tmem_ld32(c.tmem + kTmemSb + c.lane_off + kTokPer * c.th, b);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) e[j] = __uint_as_float(a[j]) + __uint_as_float(b[j]);
+        for (int j = 0; j < kTokPer; ++j) s[j] = __uint_as_float(a[j]) + __uint_as_float(b[j]);
     }
     tc_fence_before();
     __syncwarp();
     if (c.lane == 0) mbar_arrive(&sm.s_free);
-    m_own = -INFINITY;
-    if (c.warp_ok) {
-        const int k0 = key0 + 32 * c.th;
-        if (k0 + 32 > vis) {  // the sequence ends (or the causal limit falls) inside these tokens
+    const int k0 = key0 + kTokPer * c.th;
+    if (k0 + kTokPer > vis) {  // the sequence ends (or the causal limit falls) inside these tokens
 #pragma unroll
-            for (int j = 0; j < 32; ++j) e[j] = k0 + j < vis ? e[j] : -INFINITY;
-        }
-        float t[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) t[j] = fmaxf(e[j], e[j + 16]);
-#pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-            for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
-        const float sl2 = c.p->scale_log2;  // > 0, so the max commutes with the scaling
-        const bool none = t[0] == -INFINITY;
-        m_own = none ? -INFINITY : t[0] * sl2;
-        const float off = none ? 0.f : kXScaleLog2 - m_own;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) e[j] = none ? 0.f : ex2_approx(fmaf(e[j], sl2, off));
-        const int slot = g & 1;
-        const uint32_t base = c.xchg_peer + (uint32_t)(((slot * 2 + c.th) * 4) * 128 + c.i) * 16;
-        const uint32_t bar = c.xfull_peer0 + slot * 8;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            uint32_t w[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                __half2 two = __floats2half2_rn(e[8 * c4 + 2 * q], e[8 * c4 + 2 * q + 1]);
-                w[q] = *reinterpret_cast<uint32_t *>(&two);
-            }
-            st_async_v4_b32(base + c4 * 128 * 16, w[0], w[1], w[2], w[3], bar);
-        }
-        // the row offset travels in the offsets area of the same slot
-        const uint32_t offa = c.xchg_peer + (uint32_t)(2 * 2 * 4 * 128 * 16) + (uint32_t)((slot * 2 + c.th) * 128 + c.i) * 4;
-        st_async_b32(offa, __float_as_uint(m_own), bar);
+        for (int j = 0; j < kTokPer; ++j) s[j] = k0 + j < vis ? s[j] : -INFINITY;
     }
     return true;
+}
+
+// E (fp16) and m (fp32) of block g into the peer CTA's receive slot g % 2. Each thread sends
+// block g+1 only after it has consumed the peer's block g, and the peer sent block g only after
+// consuming slot (g - 1) % 2 = (g + 1) % 2 itself, so two slots never overrun.
+__device__ __forceinline__ void send_factors(const SoftCtx &c, int g, const float (&e)[kTokPer], float m_own) {
+    if (!c.warp_ok) return;
+    const int slot = g & 1;
+    const uint32_t base = c.xchg_peer + (uint32_t)(((slot * kTq + c.th) * 4) * 128 + c.i) * 16;
+    const uint32_t bar = c.xfull_peer0 + slot * 8;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            __half2 two = __floats2half2_rn(e[8 * c4 + 2 * q], e[8 * c4 + 2 * q + 1]);
+            w[q] = *reinterpret_cast<uint32_t *>(&two);
+        }
+        st_async_v4_b32(base + c4 * 128 * 16, w[0], w[1], w[2], w[3], bar);
+    }
+    // the row offset travels in the offsets area of the same slot
+    const uint32_t offa = c.xchg_peer + (uint32_t)kXchgEBytes + (uint32_t)((slot * kTq + c.th) * 128 + c.i) * 4;
+    st_async_b32(offa, __float_as_uint(m_own), bar);
+}
+
+// E = 2^(s * scale_log2 - m + 15) in place with m = max_j s_j * scale_log2 (log2 units); E is in
+// [0, 2^15], 0 for masked tokens.
+__device__ __forceinline__ float exps_in_place(float (&s)[kTokPer], float sl2) {
+    float t[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) t[j] = fmaxf(s[j], s[j + 16]);
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+    const bool none = t[0] == -INFINITY;
+    const float m = none ? -INFINITY : t[0] * sl2;  // sl2 > 0, so the max commutes with the scaling
+    const float off = none ? 0.f : kXScaleLog2 - m;
+#pragma unroll
+    for (int j = 0; j < kTokPer; ++j) s[j] = ex2_approx(fmaf(s[j], sl2, off));
+    return m;
 }
 
 __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem, uint32_t half,
@@ -415,57 +425,63 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     c.xchg_peer = map_to_rank(&sm.xchg[0], peer);
     c.xfull_peer0 = map_to_rank(&sm.xfull[0], peer);
     const int nvalid_warps = min(4, (p.rows - group * 128 + 31) / 32);
-    const uint32_t xbytes = (uint32_t)nvalid_warps * 2 * 32 * (64 + 4);  // both token halves: E (64 B) + offset
+    const uint32_t xbytes = (uint32_t)nvalid_warps * kTq * 32 * (2 * kTokPer + 4);  // E (fp16) + offset
     const int t_q = c.row_ok ? c.r / p.h_q : 0, h_idx = c.row_ok ? c.r % p.h_q : 0;
+    const float sl2 = p.scale_log2;
     volatile int *abort = &sm.abort;
-    const float4 *xe = reinterpret_cast<const float4 *>(sm.xchg);
-    const float *xo = reinterpret_cast<const float *>(sm.xchg + 2 * 2 * 4 * 128);  // offsets area
+    const uint4 *xe = sm.xchg;
+    const float *xo = reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(sm.xchg) + kXchgEBytes);
+    const int bar_id = 1 + wq;  // the two warps of these 32 rows
 
-    BlockWalker wa;
-    wa.init(meta, p);
-    if (!wa.live) return;
-    load_q(sm, c, wa.pc);
-    int vis = c.row_ok ? visible_keys(wa.pc.n, p.s_q, t_q, p.causal) : 0;
-    float e_own[32], m_own;
-    if (!load_and_send(sm, c, 0, wa.blk * kBlk, vis, e_own, m_own)) return;
-    if (wa.last()) {  // the next piece's Q may replace this one once its last Gemm1 is done
-        Cursor tmp = wa.cur;
+    // w walks one block ahead of the block being finished; of that block only a few facts are kept
+    BlockWalker w;
+    w.init(meta, p);
+    if (!w.live) return;
+    load_q(sm, c, w.pc);
+    int vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
+    float e_own[kTokPer], m_own;
+    if (!load_raw(sm, c, 0, w.blk * kBlk, vis, e_own)) return;
+    m_own = exps_in_place(e_own, sl2);
+    send_factors(c, 0, e_own, m_own);
+    if (w.last()) {  // the next piece's Q may replace this one once its last Gemm1 is done
+        Cursor tmp = w.cur;
         Piece nx;
         if (tmp.next(p, nx)) load_q(sm, c, nx);
     }
     float m_ref = -INFINITY, l = 0.f;
-    for (int g = 0; wa.live; ++g) {
-        BlockWalker wb = wa;
-        wb.advance(p);
+    for (int g = 0; w.live; ++g) {
+        const bool a_first = w.first(), a_last = w.last();
+        const int a_piece_k = w.piece_k, a_seq = w.pc.seq, a_nsplit = w.pc.nsplit, a_slot = w.pc.slot;
+        w.advance(p);
+        const bool nx_live = w.live;
+        // raw scores of block g+1 first: the accumulators are free for Gemm1 of block g+2 early, and
+        // the peer's factors of block g arrive meanwhile
+        float snx[kTokPer];
+        if (nx_live) {
+            if (w.first()) vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
+            if (!load_raw(sm, c, g + 1, w.blk * kBlk, vis, snx)) return;
+            if (w.last()) {
+                Cursor tmp = w.cur;
+                Piece nx;
+                if (tmp.next(p, nx)) load_q(sm, c, nx);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < kTokPer; ++j) snx[j] = -INFINITY;
+        }
         // peer factors of block g (slot g % 2)
         const int slot = g & 1;
         if (threadIdx.x == 32 * kFirstSoftWarp) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
         if (!mbar_wait_cluster(&sm.xfull[slot], (g >> 1) & 1, abort)) return;
-        float e_peer[32];
-        float m_peer = -INFINITY;
-        if (c.warp_ok) {
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const float4 v = xe[((slot * 2 + c.th) * 4 + c4) * 128 + c.i];
-                const uint32_t w[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
-                                       __float_as_uint(v.w)};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[q]));
-                    e_peer[8 * c4 + 2 * q] = f.x;
-                    e_peer[8 * c4 + 2 * q + 1] = f.y;
-                }
-            }
-            m_peer = xo[(slot * 2 + c.th) * 128 + c.i];
-        }
+        const float m_peer = c.warp_ok ? xo[(slot * kTq + c.th) * 128 + c.i] : -INFINITY;
         // an upper bound of the block's row max (both token halves), shared by the two warps of a row
         const float mbu_half = m_own + m_peer;
         sm.xmax[g & 1][c.th][c.i] = mbu_half;
-        named_bar_sync(1 + (c.i >> 5), 64);  // the two warps of these 32 rows
+        named_bar_sync(bar_id, 64);
         const float mbu = fmaxf(mbu_half, sm.xmax[g & 1][c.th ^ 1][c.i]);
         bool need = false;
         float alpha = 1.f;
-        if (wa.first()) {
+        if (a_first) {
             m_ref = mbu;
             l = 0.f;
         } else if (mbu > m_ref + kRescaleThreshold) {
@@ -478,44 +494,50 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 need = true;
             }
         }
+        uint32_t ep[kTokPer / 2];  // the peer's factors, fp16 pairs
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 v = xe[((slot * kTq + c.th) * 4 + c4) * 128 + c.i];
+            ep[4 * c4] = v.x;
+            ep[4 * c4 + 1] = v.y;
+            ep[4 * c4 + 2] = v.z;
+            ep[4 * c4 + 3] = v.w;
+        }
+        // One straight-line region: P of block g (FMA and ALU work) and the exponentials of block
+        // g+1 (MUFU work), so that the scheduler can overlap the two.
         // P = 2^(s0 + s1 - m_ref) in two bf16 terms: hi = P with its low 16 bits cleared, lo = the
         // (exact) remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P.
-        uint32_t pk[16], pl[16];
-        if (c.warp_ok) {
-            const bool none = m_ref == -INFINITY || mbu_half == -INFINITY;
-            const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 2.f * kXScaleLog2);
-            float su[4] = {0.f, 0.f, 0.f, 0.f};
+        const bool none = m_ref == -INFINITY || mbu_half == -INFINITY;
+        const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 2.f * kXScaleLog2);
+        const float m_nx = exps_in_place(snx, sl2);  // unused when there is no block g+1
+        uint32_t pk[kTokPer / 2], pl[kTokPer / 2];
+        float su[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const float p0 = e_own[j] * e_peer[j] * f, p1 = e_own[j + 1] * e_peer[j + 1] * f;
-                su[(j >> 1) & 3] += p0 + p1;
-                const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-                const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
-                pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
-                pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
-            }
-            l += (su[0] + su[1]) + (su[2] + su[3]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) pk[j] = pl[j] = 0u;
+        for (int j = 0; j < kTokPer; j += 2) {
+            const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
+            const float p0 = e_own[j] * e2.x * f, p1 = e_own[j + 1] * e2.y * f;
+            su[(j >> 1) & 3] += p0 + p1;
+            const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+            const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+            pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
+            pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
         }
+        l += (su[0] + su[1]) + (su[2] + su[3]);
         // the P tile and O are free once Gemm2 of block g-1 has completed
         if (g > 0 && !mbar_wait(&sm.p_free, (g - 1) & 1, abort)) return;
         tc_fence_after();
-        if (c.warp_ok) {
-            if (__any_sync(0xffffffffu, need)) {
-                const float a = need ? alpha : 1.f;
+        if (c.warp_ok && __any_sync(0xffffffffu, need)) {
+            const float a = need ? alpha : 1.f;
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + kTmemO + c.lane_off + 128 * c.th + 32 * q, v);
-                    tmem_wait_ld();
+            for (int q = 0; q < 8; ++q) {
+                uint32_t v[16];
+                tmem_ld16(tmem + kTmemO + c.lane_off + 128 * c.th + 16 * q, v);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * a);
-                    tmem_st32(tmem + kTmemO + c.lane_off + 128 * c.th + 32 * q, v);
-                }
-                tmem_wait_st();
+                for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * a);
+                tmem_st16(tmem + kTmemO + c.lane_off + 128 * c.th + 16 * q, v);
             }
+            tmem_wait_st();
         }
         {  // this thread's 64 bytes of row i in both P tiles (K-major, 128-byte swizzle)
             uint8_t *row_hi = sm.p_tile[0] + c.i * 128, *row_lo = sm.p_tile[1] + c.i * 128;
@@ -531,44 +553,45 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         __syncwarp();
         if (c.lane == 0) mbar_arrive(&sm.p_full);
 
-        if (wa.last()) {  // epilogue of this piece: the two token halves' sums, then this warp's O columns
-            sm.xsum[c.th][c.i] = l;
-            named_bar_sync(1 + (c.i >> 5), 64);
-            const float l_row = l + sm.xsum[c.th ^ 1][c.i];
-            if (!mbar_wait(&sm.o_full, wa.piece_k & 1, abort)) return;
+        if (a_last) {  // epilogue of this piece: the two token halves' sums, then this warp's O columns
+            // the sums travel in the other parity's row-max slots, which nobody reads until block g+1
+            sm.xmax[(g + 1) & 1][c.th][c.i] = l;
+            named_bar_sync(bar_id, 64);
+            const float l_row = l + sm.xmax[(g + 1) & 1][c.th ^ 1][c.i];
+            named_bar_sync(bar_id, 64);  // both sums read before block g+1 reuses the slots
+            if (!mbar_wait(&sm.o_full, a_piece_k & 1, abort)) return;
             tc_fence_after();
             if (c.warp_ok) {
-                const Piece &cp = wa.pc;
                 const bool empty = !(l_row > 0.f);
                 const float inv = empty ? 0.f : 1.f / l_row;
-                const bool whole = cp.nsplit == 1;
+                const bool whole = a_nsplit == 1;
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t v[32];
-                    const int col = 128 * c.th + 32 * q;
-                    tmem_ld32(tmem + kTmemO + c.lane_off + col, v);
+                for (int q = 0; q < 8; ++q) {
+                    uint32_t v[16];
+                    const int col = 128 * c.th + 16 * q;
+                    tmem_ld16(tmem + kTmemO + c.lane_off + col, v);
                     tmem_wait_ld();
                     if (!c.row_ok) continue;
                     if (whole) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)cp.seq * p.rows + c.r) * kDv +
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)a_seq * p.rows + c.r) * kDv +
                                                                256 * half + col);
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint32_t w[4];
+                        for (int q4 = 0; q4 < 2; ++q4) {
+                            uint32_t wv[4];
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 __nv_bfloat162 two =
                                     __floats2bfloat162_rn(__uint_as_float(v[8 * q4 + 2 * j]) * inv,
                                                           __uint_as_float(v[8 * q4 + 2 * j + 1]) * inv);
-                                w[j] = *reinterpret_cast<uint32_t *>(&two);
+                                wv[j] = *reinterpret_cast<uint32_t *>(&two);
                             }
-                            dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+                            dst[q4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                         }
                     } else {
-                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((size_t)cp.slot * p.rows + c.r) * kDv +
+                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((size_t)a_slot * p.rows + c.r) * kDv +
                                                                  256 * half + col);
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4)
+                        for (int q4 = 0; q4 < 4; ++q4)
                             dst[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
                                                   __uint_as_float(v[4 * q4 + 2]) * inv,
                                                   __uint_as_float(v[4 * q4 + 3]) * inv);
@@ -577,26 +600,21 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 if (c.row_ok && half == 0 && c.th == 0) {
                     const float lse = empty ? -INFINITY : (m_ref + log2f(l_row)) * 0.69314718055994530942f;
                     if (whole)
-                        p.lse[((size_t)cp.seq * p.h_q + h_idx) * p.s_q + t_q] = lse;
+                        p.lse[((size_t)a_seq * p.h_q + h_idx) * p.s_q + t_q] = lse;
                     else
-                        p.lse_part[(size_t)cp.slot * p.rows + c.r] = lse;
+                        p.lse_part[(size_t)a_slot * p.rows + c.r] = lse;
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (c.lane == 0) mbar_arrive(&sm.o_free);
         }
-        // scores of block g+1 (frees the accumulators for Gemm1 of block g+2)
-        if (wb.live) {
-            if (wb.first()) vis = c.row_ok ? visible_keys(wb.pc.n, p.s_q, t_q, p.causal) : 0;
-            if (!load_and_send(sm, c, g + 1, wb.blk * kBlk, vis, e_own, m_own)) return;
-            if (wb.last()) {
-                Cursor tmp = wb.cur;
-                Piece nx;
-                if (tmp.next(p, nx)) load_q(sm, c, nx);
-            }
+        if (nx_live) {
+            send_factors(c, g + 1, snx, m_nx);
+#pragma unroll
+            for (int j = 0; j < kTokPer; ++j) e_own[j] = snx[j];
+            m_own = m_nx;
         }
-        wa = wb;
     }
 }
 
@@ -617,14 +635,14 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
         }
-        mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.s_free, 8);
-        mbar_init(&sm.p_full, 8);
+        mbar_init(&sm.s_full, 2);
+        mbar_init(&sm.s_free, kSoftWarps);
+        mbar_init(&sm.p_full, kSoftWarps);
         mbar_init(&sm.p_free, 1);
         mbar_init(&sm.o_full, 1);
-        mbar_init(&sm.o_free, 8);
-        mbar_init(&sm.q_full, 8);
-        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.o_free, kSoftWarps);
+        mbar_init(&sm.q_full, kSoftWarps);
+        mbar_init(&sm.mma_done, 3);
         mbar_init(&sm.xfull[0], 1);
         mbar_init(&sm.xfull[1], 1);
         sm.abort = 0;
@@ -644,8 +662,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
         setmaxnreg_dec<kRegsControl>();
         if (warp == 0) {
             if (lane == 0) producer(sm, p, &map_lat, &map_rope, meta, half);
-        } else if (warp == 1) {
-            mma_warp(sm, p, meta, tmem);
+        } else {
+            if (warp == 3)
+                gemm2_warp(sm, p, meta, tmem);
+            else
+                gemm1_warp(sm, p, meta, tmem, warp - 1);
+            drain_mmas(sm);
         }
     } else {
         setmaxnreg_inc<kRegsSoftmax>();

@@ -55,11 +55,29 @@ MLA_DEV bool mbar_test_cluster(uint64_t *bar, uint32_t parity) {
 
 // Bounded wait for phase `parity`. Gives up (returns false) when *abort is set by another
 // role or when the clock budget runs out (then it sets *abort itself).
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes (or the hint
+// runs out) instead of spinning, so waiting warps leave the issue slots to the working ones.
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms
+MLA_DEV bool mbar_sleep_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs) : "memory");
+    return ok != 0;
+}
+MLA_DEV bool mbar_sleep_test_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs) : "memory");
+    return ok != 0;
+}
 MLA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_test(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_test(bar, parity)) return true;
+        if (mbar_sleep_test(bar, parity)) return true;
         if (*abort) return false;
         if (clock64() - t0 > kSpinCycles) {
             *abort = 1;
@@ -71,7 +89,7 @@ MLA_DEV bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abo
     if (mbar_test_cluster(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_test_cluster(bar, parity)) return true;
+        if (mbar_sleep_test_cluster(bar, parity)) return true;
         if (*abort) return false;
         if (clock64() - t0 > kSpinCycles) {
             *abort = 1;
@@ -149,6 +167,13 @@ MLA_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+MLA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
 MLA_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
