@@ -365,9 +365,8 @@ __device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int 
     return true;
 }
 
-// E (fp16) and m (fp32) of block g into the peer CTA's receive slot g % 2. Each thread sends
-// block g+1 only after it has consumed the peer's block g, and the peer sent block g only after
-// consuming slot (g - 1) % 2 = (g + 1) % 2 itself, so two slots never overrun.
+// E (fp16) and m (fp32) of block g into the peer CTA's receive slot g % 2 (the first block of a
+// part; later blocks are sent from the softmax loop as their exponentials are computed).
 __device__ __forceinline__ void send_factors(const SoftCtx &c, int g, const float (&e)[kTokPer], float m_own) {
     if (!c.warp_ok) return;
     const int slot = g & 1;
@@ -424,6 +423,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     const uint32_t peer = half ^ 1u;
     c.xchg_peer = map_to_rank(&sm.xchg[0], peer);
     c.xfull_peer0 = map_to_rank(&sm.xfull[0], peer);
+    const uint32_t xchg_peer = c.xchg_peer, xfull_peer0 = c.xfull_peer0;
     const int nvalid_warps = min(4, (p.rows - group * 128 + 31) / 32);
     const uint32_t xbytes = (uint32_t)nvalid_warps * kTq * 32 * (2 * kTokPer + 4);  // E (fp16) + offset
     const int t_q = c.row_ok ? c.r / p.h_q : 0, h_idx = c.row_ok ? c.r % p.h_q : 0;
@@ -503,25 +503,59 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
             ep[4 * c4 + 2] = v.z;
             ep[4 * c4 + 3] = v.w;
         }
-        // One straight-line region: P of block g (FMA and ALU work) and the exponentials of block
-        // g+1 (MUFU work), so that the scheduler can overlap the two.
+        // One straight-line region: P of block g (FMA and ALU work), the exponentials of block g+1
+        // (MUFU work) and their stores into the peer (distributed shared memory, ~20 bytes per
+        // cycle), spread over the region so that the three overlap. Sending block g+1 here is safe
+        // with two receive slots: the peer sent block g (which has arrived) only after it had read
+        // slot (g - 1) % 2 = (g + 1) % 2.
         // P = 2^(s0 + s1 - m_ref) in two bf16 terms: hi = P with its low 16 bits cleared, lo = the
         // (exact) remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P.
         const bool none = m_ref == -INFINITY || mbu_half == -INFINITY;
         const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 2.f * kXScaleLog2);
-        const float m_nx = exps_in_place(snx, sl2);  // unused when there is no block g+1
+        float m_nx, off_nx;
+        {
+            float t[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) t[j] = fmaxf(snx[j], snx[j + 16]);
+#pragma unroll
+            for (int k = 8; k >= 1; k >>= 1)
+#pragma unroll
+                for (int j = 0; j < k; ++j) t[j] = fmaxf(t[j], t[j + k]);
+            const bool nx_none = t[0] == -INFINITY;
+            m_nx = nx_none ? -INFINITY : t[0] * sl2;  // sl2 > 0, so the max commutes with the scaling
+            off_nx = nx_none ? 0.f : kXScaleLog2 - m_nx;
+        }
+        const bool send = nx_live && c.warp_ok;
+        const int nslot = (g + 1) & 1;
+        const uint32_t xbase = xchg_peer + (uint32_t)(((nslot * kTq + c.th) * 4) * 128 + c.i) * 16;
+        const uint32_t xbar = xfull_peer0 + nslot * 8;
         uint32_t pk[kTokPer / 2], pl[kTokPer / 2];
         float su[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < kTokPer; j += 2) {
-            const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
-            const float p0 = e_own[j] * e2.x * f, p1 = e_own[j + 1] * e2.y * f;
-            su[(j >> 1) & 3] += p0 + p1;
-            const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-            const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
-            pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
-            pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+        for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int j = 8 * c4 + 2 * q;
+                // E of block g+1: 2^(s * scale_log2 - m + 15), in [0, 2^15], 0 for masked tokens
+                snx[j] = ex2_approx(fmaf(snx[j], sl2, off_nx));
+                snx[j + 1] = ex2_approx(fmaf(snx[j + 1], sl2, off_nx));
+                __half2 two = __floats2half2_rn(snx[j], snx[j + 1]);
+                wv[q] = *reinterpret_cast<uint32_t *>(&two);
+                // P of block g
+                const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
+                const float p0 = e_own[j] * e2.x * f, p1 = e_own[j + 1] * e2.y * f;
+                su[q] += p0 + p1;
+                const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
+                pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+            }
+            if (send) st_async_v4_b32(xbase + c4 * 128 * 16, wv[0], wv[1], wv[2], wv[3], xbar);
         }
+        if (send)  // the row offset travels in the offsets area of the same slot
+            st_async_b32(xchg_peer + (uint32_t)kXchgEBytes + (uint32_t)((nslot * kTq + c.th) * 128 + c.i) * 4,
+                         __float_as_uint(m_nx), xbar);
         l += (su[0] + su[1]) + (su[2] + su[3]);
         // the P tile and O are free once Gemm2 of block g-1 has completed
         if (g > 0 && !mbar_wait(&sm.p_free, (g - 1) & 1, abort)) return;
@@ -610,7 +644,6 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
             if (c.lane == 0) mbar_arrive(&sm.o_free);
         }
         if (nx_live) {
-            send_factors(c, g + 1, snx, m_nx);
 #pragma unroll
             for (int j = 0; j < kTokPer; ++j) e_own[j] = snx[j];
             m_own = m_nx;
