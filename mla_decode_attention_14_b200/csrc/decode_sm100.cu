@@ -15,34 +15,34 @@
 //    [256h, 256h+256) and rotary dims [512+32h, 512+32h+32), i.e. exactly half of every block
 //    (36,864 bytes); the pair together reads each block once.
 //  * Gemm1 is split along its 576-long contraction: CTA h computes the partial scores over its
-//    288 dims (18 tcgen05 MMAs, M=128 rows, N=64 tokens, into two accumulators of 9 k-steps each
-//    so that consecutive MMAs do not wait on one another; the latent part of Q is the A operand
-//    in TMEM, the rotary part in shared memory).
+//    288 dims (18 tcgen05 MMAs, M=128 rows, N=64 tokens, into one accumulator; the latent part
+//    of Q is the A operand in TMEM, the rotary part in shared memory).
 //  * The pair combines the partial scores multiplicatively: 2^(s0 + s1 - m) =
 //    2^(s0 - m0) * 2^(s1 - m1) * 2^(m0 + m1 - m). Each CTA computes E = 2^(s - m + 15) for its
 //    own partial with its own row offset m, keeps it in fp32, and sends it to the peer as fp16
 //    together with m in fp32: st.async stores into the peer's 2-slot receive ring complete on
 //    the peer's mbarrier. E lies in (0, 2^15], so the exchanged factor keeps fp16's relative
 //    precision (2^-11) down to 2^-29 of the row max whatever the score magnitude, and the
-//    traffic is half that of fp32 scores.
+//    traffic is half that of fp32 scores. The link between the two SMs moves only about 20
+//    bytes per cycle, so the stores are spread over the softmax warps' compute.
 //  * Eight softmax warps: warp w serves TMEM lane quarter w&3 (32 query rows) and one half of
 //    every block's tokens; the two halves of a row agree on an upper bound of the block max
 //    through shared memory, so both take the same lazy-rescaling decisions (O is rescaled only
 //    when the running max grows by more than 2^8). P = E_own * E_peer * 2^(m0 + m1 - m - 30) goes
-//    to shared memory as two bf16 terms (hi = P with its low 16 bits cleared, lo = the exact
-//    remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P), so P's rounding
-//    does not add to the bf16 output rounding.
-//  * Issuing a tcgen05 MMA occupies the issuing thread for about 70 cycles, so three warps issue:
-//    one per Gemm1 accumulator and one for Gemm2. The softmax warps read the scores of block g+1
-//    before they finish block g, so Gemm1 of block g+2 can start while Gemm2 of block g waits for P.
-//  * Gemm2: 8 MMAs (M=128, N=256, K=16 tokens; A = P_hi then P_lo, K-major in shared memory,
-//    B = the value half of the same cache tile read MN-major): the block is loaded once for
-//    both GEMMs.
-//  * Warp roles: warp 0 lane 0 = TMA producer (4-stage ring, block-table gather, L2
-//    evict-first); warps 1-2 issue Gemm1 (warp 1 also owns the TMEM allocation); warp 3 issues
-//    Gemm2 and zeroes the cache rows past a sequence's end before Gemm2 reads them, so undefined
-//    tail contents never reach the result; warps 4-11 = softmax, correction and epilogue (a warp
-//    may only touch TMEM lane quarter w & 3). Warpgroup 0 hands registers to the softmax warps.
+//    to TMEM as two bf16 terms (hi = P with its low 16 bits cleared, lo = the exact remainder
+//    with its low 16 bits cleared; hi + lo is within 2^-14 of P), so P's rounding does not add
+//    to the bf16 output rounding.
+//  * Issuing a tcgen05 MMA occupies the issuing thread for about 70 cycles, so Gemm1 and Gemm2
+//    have their own issuing warps and the tensor core runs both at once. The softmax warps read
+//    the scores of block g+1 before they finish block g, so Gemm1 of block g+2 runs while
+//    Gemm2 of block g waits for P.
+//  * Gemm2: 8 MMAs (M=128, N=256, K=16 tokens; A = P_hi then P_lo from TMEM, B = the value half
+//    of the same cache tile read MN-major): the block is loaded once for both GEMMs.
+//  * Warp roles: warp 0 lane 0 = TMA producer (5-stage ring, block-table gather, L2
+//    evict-first); warp 1 issues Gemm1 and owns the TMEM allocation; warp 3 issues Gemm2 and
+//    zeroes the cache rows past a sequence's end before Gemm2 reads them, so undefined tail
+//    contents never reach the result; warps 4-11 = softmax, correction and epilogue (a warp may
+//    only touch TMEM lane quarter w & 3). Warpgroup 0 hands registers to the softmax warps.
 //  * Pieces of split sequences leave fp32 partial O and lse in the workspace for the combine
 //    kernel; whole sequences are written straight to bf16 out / fp32 lse.
 // Every wait is bounded; a timeout sets the device error word and the CTA exits cleanly.
@@ -55,7 +55,7 @@ namespace mla {
 using namespace sm100;
 
 namespace dec {
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kFirstSoftWarp = 4;                 // warpgroup 0: TMA producer and the three MMA-issuing warps
 constexpr int kSoftWarps = 8;                     // two per SM sub-partition
 constexpr int kThreads = 32 * (kFirstSoftWarp + kSoftWarps);  // 384
@@ -75,16 +75,15 @@ constexpr float kXScaleLog2 = 15.0f;
 // TMEM column map (512 columns allocated, 128 lanes = 128 query rows)
 constexpr uint32_t kTmemO = 0;     // 256 fp32: O for this CTA's 256 value dims
 constexpr uint32_t kTmemQ = 256;   // 128 x (2 bf16): this CTA's 256 latent query dims
-constexpr uint32_t kTmemSa = 384;  // 64 fp32: partial scores, first half of the k-steps
-constexpr uint32_t kTmemSb = 448;  // 64 fp32: partial scores, second half of the k-steps
+constexpr uint32_t kTmemS = 384;   // 64 fp32: partial scores of a block
+constexpr uint32_t kTmemPhi = 448; // 32 x (2 bf16): P with its low 16 bits cleared (the A operand of Gemm2)
+constexpr uint32_t kTmemPlo = 480; // 32 x (2 bf16): the remainder, likewise
 constexpr uint32_t kTmemCols = 512;
-constexpr int kPTileBytes = 128 * 128;  // 128 rows x 64 tokens bf16, K-major, 128-byte swizzle
 constexpr int kXchgEBytes = 2 * kBlk * 128 * 2;    // two slots of 128 rows x 64 fp16 factors
 constexpr int kXchgOffBytes = 2 * kTq * 128 * 4;   // two slots of 128 rows x 2 fp32 offsets
 
 struct __align__(1024) Smem {
     uint8_t stage[kStages][kStageBytes];  // KV ring
-    uint8_t p_tile[2][kPTileBytes];       // P of the current block: [0] = bf16 high part, [1] = low part
     uint4 xchg[(kXchgEBytes + kXchgOffBytes) / 16];  // peer E factors (fp16) [slot][token half][16 B][row]
                                                      // + row offsets (fp32) [slot][token half][row]
     float xmax[2][kTq][128];  // per-row exchange between the two token halves (block max bound; sums)
@@ -218,16 +217,14 @@ __device__ void zero_tail_rows(uint8_t *st, int valid, int lane) {
 }
 
 // Issuing one tcgen05 MMA occupies the issuing thread for about 70 cycles whatever its size, so
-// the small Gemm1 MMAs (N = 64) are spread over two issuing warps, one per accumulator, and
-// Gemm2 has a third: the tensor core takes MMAs from all three at once.
+// Gemm1 and Gemm2 are issued by two warps: the tensor core takes MMAs from both at once.
 
-// Gemm1 of every block into accumulator `which` (0: latent k-steps 0-7 + rotary k-step 0 into S_a,
-// 1: latent k-steps 8-15 + rotary k-step 1 into S_b); s_full completes once both have landed.
-__device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem, int which) {
+// Gemm1 of every block into S (partial scores over this CTA's 288 dims): 18 MMAs into one
+// accumulator; the next block's Gemm1 may start as soon as the softmax warps have read S.
+__device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
     constexpr uint32_t id1 = idesc_bf16_f32(128, 64, 0);  // S = Q K^T: K-major B
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
-    const uint32_t d = tmem + (which ? kTmemSb : kTmemSa);
     BlockWalker w;
     w.init(meta, p);
     for (int g = 0; w.live; w.advance(p), ++g) {
@@ -242,12 +239,12 @@ __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
             const uint64_t rd = smem_desc(smem_addr(sm.stage[s]) + 4 * kBoxBytes, 16, 512, 4);
             const uint64_t qd = smem_desc(smem_addr(sm.q_rope), 16, 512, 4);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {  // latent k-steps, A (Q) from TMEM
-                const int kk = 8 * which + k;
-                mma_ts(d, tmem + kTmemQ + 8 * kk, kd + (uint64_t)(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4), id1,
-                       k > 0 ? 1u : 0u);
-            }
-            mma_ss(d, qd + 2 * which, rd + 2 * which, id1, 1u);  // rotary k-step, A from shared memory
+            for (int k = 0; k < 16; ++k)  // latent k-steps, A (Q) from TMEM
+                mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * k, kd + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4),
+                       id1, k > 0 ? 1u : 0u);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)  // rotary k-steps, A from shared memory
+                mma_ss(tmem + kTmemS, qd + 2 * c, rd + 2 * c, id1, 1u);
             mma_commit(&sm.s_full);
         }
         __syncwarp();
@@ -270,13 +267,12 @@ __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
         if (lane == 0) {
             tc_fence_after();
             const uint64_t vd = smem_desc(smem_addr(sm.stage[s]), 4 * 2048, 1024, 2);
-            const uint64_t pd = smem_desc(smem_addr(sm.p_tile[0]), 16, 1024, 2);
             const bool first = w.first();
 #pragma unroll
-            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo, both K-major in shared memory
+            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo, A from TMEM
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tmem + kTmemO, pd + (uint64_t)((hl * kPTileBytes + 32 * kk) >> 4), vd + 128 * kk, id2,
+                    mma_ts(tmem + kTmemO, tmem + (hl ? kTmemPlo : kTmemPhi) + 8 * kk, vd + 128 * kk, id2,
                            (!first || hl > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&sm.p_free);
             mma_commit(&sm.kv_empty[s]);
@@ -347,12 +343,11 @@ __device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int 
     if (!mbar_wait(&sm.s_full, g & 1, &sm.abort)) return false;
     tc_fence_after();
     {
-        uint32_t a[32], b[32];
-        tmem_ld32(c.tmem + kTmemSa + c.lane_off + kTokPer * c.th, a);
-        tmem_ld32(c.tmem + kTmemSb + c.lane_off + kTokPer * c.th, b);
+        uint32_t a[32];
+        tmem_ld32(c.tmem + kTmemS + c.lane_off + kTokPer * c.th, a);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < kTokPer; ++j) s[j] = __uint_as_float(a[j]) + __uint_as_float(b[j]);
+        for (int j = 0; j < kTokPer; ++j) s[j] = __uint_as_float(a[j]);
     }
     tc_fence_before();
     __syncwarp();
@@ -573,16 +568,10 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
             }
             tmem_wait_st();
         }
-        {  // this thread's 64 bytes of row i in both P tiles (K-major, 128-byte swizzle)
-            uint8_t *row_hi = sm.p_tile[0] + c.i * 128, *row_lo = sm.p_tile[1] + c.i * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int chunk = ((4 * c.th + q) ^ (c.i & 7)) * 16;
-                *reinterpret_cast<uint4 *>(row_hi + chunk) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                *reinterpret_cast<uint4 *>(row_lo + chunk) = make_uint4(pl[4 * q], pl[4 * q + 1], pl[4 * q + 2], pl[4 * q + 3]);
-            }
-            fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
-        }
+        // this thread's 32 tokens of row i in both P regions of TMEM (bf16 pairs, lane = row)
+        tmem_st16(tmem + kTmemPhi + c.lane_off + 16 * c.th, pk);
+        tmem_st16(tmem + kTmemPlo + c.lane_off + 16 * c.th, pl);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (c.lane == 0) mbar_arrive(&sm.p_full);
@@ -668,14 +657,14 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
         }
-        mbar_init(&sm.s_full, 2);
+        mbar_init(&sm.s_full, 1);
         mbar_init(&sm.s_free, kSoftWarps);
         mbar_init(&sm.p_full, kSoftWarps);
         mbar_init(&sm.p_free, 1);
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.o_free, kSoftWarps);
         mbar_init(&sm.q_full, kSoftWarps);
-        mbar_init(&sm.mma_done, 3);
+        mbar_init(&sm.mma_done, 2);
         mbar_init(&sm.xfull[0], 1);
         mbar_init(&sm.xfull[1], 1);
         sm.abort = 0;
@@ -696,11 +685,13 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
         if (warp == 0) {
             if (lane == 0) producer(sm, p, &map_lat, &map_rope, meta, half);
         } else {
-            if (warp == 3)
+            if (warp == 3) {
                 gemm2_warp(sm, p, meta, tmem);
-            else
-                gemm1_warp(sm, p, meta, tmem, warp - 1);
-            drain_mmas(sm);
+                drain_mmas(sm);
+            } else if (warp == 1) {
+                gemm1_warp(sm, p, meta, tmem);
+                drain_mmas(sm);
+            }
         }
     } else {
         setmaxnreg_inc<kRegsSoftmax>();
