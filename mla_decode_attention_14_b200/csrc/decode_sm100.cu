@@ -18,17 +18,20 @@
 //    288 dims (18 tcgen05 MMAs, M=128 rows, N=64 tokens, into one accumulator; the latent part
 //    of Q is the A operand in TMEM, the rotary part in shared memory).
 //  * The pair combines the partial scores multiplicatively: 2^(s0 + s1 - m) =
-//    2^(s0 - m0) * 2^(s1 - m1) * 2^(m0 + m1 - m). Each CTA computes E = 2^(s - m + 15) for its
-//    own partial with its own row offset m, keeps it in fp32, and sends it to the peer as fp16
-//    together with m in fp32: st.async stores into the peer's 2-slot receive ring complete on
-//    the peer's mbarrier. E lies in (0, 2^15], so the exchanged factor keeps fp16's relative
-//    precision (2^-11) down to 2^-29 of the row max whatever the score magnitude, and the
-//    traffic is half that of fp32 scores. The link between the two SMs moves only about 20
-//    bytes per cycle, so the stores are spread over the softmax warps' compute.
+//    2^(s0 - m0) * 2^(s1 - m1) * 2^(m0 + m1 - m). Each CTA computes, for its own partial with
+//    its own row offset m, R = 2^((s - m)/2 + 15) -- the square root of its factor, scaled --
+//    keeps it in fp32, and sends it to the peer as fp16 together with m in fp32: st.async
+//    stores into the peer's 2-slot receive ring complete on the peer's mbarrier. R lies in
+//    [0, 2^15] and is normal in fp16 while s - m >= -58, so the exchange keeps a relative
+//    precision of 2^-10 (once squared) over 58 octaves of partial score whatever the score
+//    magnitude (rows whose two partial maxima overstate the true maximum by up to ~34 octaves
+//    lose nothing), and the traffic is half that of fp32 scores. The link between the two SMs
+//    moves only about 20 bytes per cycle, so the stores are spread over the softmax warps'
+//    compute.
 //  * Eight softmax warps: warp w serves TMEM lane quarter w&3 (32 query rows) and one half of
 //    every block's tokens; the two halves of a row agree on an upper bound of the block max
 //    through shared memory, so both take the same lazy-rescaling decisions (O is rescaled only
-//    when the running max grows by more than 2^8). P = E_own * E_peer * 2^(m0 + m1 - m - 30) goes
+//    when the running max grows by more than 2^8). P = (R_own R_peer)^2 2^(m0 + m1 - m - 60) goes
 //    to TMEM as two bf16 terms (hi = P with its low 16 bits cleared, lo = the exact remainder
 //    with its low 16 bits cleared; hi + lo is within 2^-14 of P), so P's rounding does not add
 //    to the bf16 output rounding.
@@ -68,8 +71,10 @@ constexpr int kBoxBytes = kBlk * 128;                      // 64 tokens x 64 bf1
 constexpr int kRopeBoxBytes = kBlk * 64;                   // 64 tokens x 32 bf16 (64-byte swizzle)
 constexpr int kStageBytes = 4 * kBoxBytes + kRopeBoxBytes;  // 36,864: half of one cache block
 constexpr float kRescaleThreshold = 8.0f;                  // log2 units: rescale O when max grows > 2^8
-// The factors E = 2^(s - m + 15) <= 2^15 (< 65504) cross the cluster as fp16, normal (full 11-bit
-// precision) down to 2^-29 of the row max; P folds the two 2^15 back out.
+// The pair exchanges R = 2^((s - m) / 2 + 15), the square root of a factor, in fp16: R <= 2^15
+// (< 65504), normal (full 11-bit precision) while s - m >= -58 and subnormal down to -78, so the
+// exchange spans 58 octaves of score range at a relative precision of 2^-10 once squared (a
+// factor sent directly would span only 29). P = (R_own R_peer)^2 2^(m0 + m1 - m_ref - 60).
 constexpr float kXScaleLog2 = 15.0f;
 
 // TMEM column map (512 columns allocated, 128 lanes = 128 query rows)
@@ -382,8 +387,8 @@ __device__ __forceinline__ void send_factors(const SoftCtx &c, int g, const floa
     st_async_b32(offa, __float_as_uint(m_own), bar);
 }
 
-// E = 2^(s * scale_log2 - m + 15) in place with m = max_j s_j * scale_log2 (log2 units); E is in
-// [0, 2^15], 0 for masked tokens.
+// R = 2^((s * scale_log2 - m) / 2 + 15) in place with m = max_j s_j * scale_log2 (log2 units); R
+// is in [0, 2^15], 0 for masked tokens.
 __device__ __forceinline__ float exps_in_place(float (&s)[kTokPer], float sl2) {
     float t[16];
 #pragma unroll
@@ -394,9 +399,10 @@ __device__ __forceinline__ float exps_in_place(float (&s)[kTokPer], float sl2) {
         for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
     const bool none = t[0] == -INFINITY;
     const float m = none ? -INFINITY : t[0] * sl2;  // sl2 > 0, so the max commutes with the scaling
-    const float off = none ? 0.f : kXScaleLog2 - m;
+    const float off = none ? 0.f : kXScaleLog2 - 0.5f * m;
+    const float hsl2 = 0.5f * sl2;
 #pragma unroll
-    for (int j = 0; j < kTokPer; ++j) s[j] = ex2_approx(fmaf(s[j], sl2, off));
+    for (int j = 0; j < kTokPer; ++j) s[j] = ex2_approx(fmaf(s[j], hsl2, off));
     return m;
 }
 
@@ -506,7 +512,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         // P = 2^(s0 + s1 - m_ref) in two bf16 terms: hi = P with its low 16 bits cleared, lo = the
         // (exact) remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P.
         const bool none = m_ref == -INFINITY || mbu_half == -INFINITY;
-        const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 2.f * kXScaleLog2);
+        const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 4.f * kXScaleLog2);
         float m_nx, off_nx;
         {
             float t[16];
@@ -518,7 +524,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 for (int j = 0; j < k; ++j) t[j] = fmaxf(t[j], t[j + k]);
             const bool nx_none = t[0] == -INFINITY;
             m_nx = nx_none ? -INFINITY : t[0] * sl2;  // sl2 > 0, so the max commutes with the scaling
-            off_nx = nx_none ? 0.f : kXScaleLog2 - m_nx;
+            off_nx = nx_none ? 0.f : kXScaleLog2 - 0.5f * m_nx;
         }
         const bool send = nx_live && c.warp_ok;
         const int nslot = (g + 1) & 1;
@@ -532,14 +538,15 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int j = 8 * c4 + 2 * q;
-                // E of block g+1: 2^(s * scale_log2 - m + 15), in [0, 2^15], 0 for masked tokens
-                snx[j] = ex2_approx(fmaf(snx[j], sl2, off_nx));
-                snx[j + 1] = ex2_approx(fmaf(snx[j + 1], sl2, off_nx));
+                // R of block g+1: 2^((s * scale_log2 - m) / 2 + 15), in [0, 2^15], 0 for masked tokens
+                snx[j] = ex2_approx(fmaf(snx[j], 0.5f * sl2, off_nx));
+                snx[j + 1] = ex2_approx(fmaf(snx[j + 1], 0.5f * sl2, off_nx));
                 __half2 two = __floats2half2_rn(snx[j], snx[j + 1]);
                 wv[q] = *reinterpret_cast<uint32_t *>(&two);
                 // P of block g
                 const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
-                const float p0 = e_own[j] * e2.x * f, p1 = e_own[j + 1] * e2.y * f;
+                const float t0 = e_own[j] * e2.x, t1 = e_own[j + 1] * e2.y;
+                const float p0 = t0 * t0 * f, p1 = t1 * t1 * f;
                 su[q] += p0 + p1;
                 const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
                 const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);

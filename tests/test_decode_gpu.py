@@ -49,6 +49,37 @@ def test_small_shapes_parity(case):
     parity.full_parity(inp, num_parts=parts, what=str(case))
 
 
+def test_maximum_rows_parity():
+    """s_q * h_q at the library's limit (1024 rows = 8 groups of 128), causal, a ragged batch."""
+    h_q, s_q = 128, 8
+    assert h_q * s_q == 1024  # MLA_MAX_ROWS in include/mla.h
+    wl = W.custom(3, h_q, s_q, [300, 70, 9], causal=True)
+    inp = W.make_inputs(wl, seed=11, tail="nan", spare_blocks=1)
+    parity.full_parity(inp, what="1024 rows")
+
+
+@pytest.mark.parametrize("scale", [0.6, 0.3, 0.01])
+def test_other_scales_parity(scale):
+    """Scales away from 192^-0.5. At 0.6, N(0,1) inputs give scores with a standard deviation of 14
+    (21 octaves), so each CTA's partial scores span ~70 octaves and the two partial maxima
+    overstate the true maximum by ~20: most of the range the pair's factor exchange covers (its
+    square-root fp16 encoding is exact to 2^-10 over 58 octaves below a thread's partial maximum).
+    0.01 makes the softmax nearly uniform."""
+    wl = W.custom(3, 64, 1, [1000, 64, 333], scale=scale)
+    inp = W.make_inputs(wl, seed=5, tail="nan")
+    parity.full_parity(inp, num_parts=5, what="scale %g" % scale)
+
+
+def test_many_short_sequences_parity():
+    """A batch of 700 short sequences of random lengths (0 to 200, some empty): many pieces per part."""
+    rng = np.random.default_rng(17)
+    seqlens = rng.integers(0, 201, size=700)
+    seqlens[::97] = 0
+    wl = W.custom(len(seqlens), 16, 1, seqlens)
+    inp = W.make_inputs(wl, seed=6, tail="nan")
+    parity.full_parity(inp, what="700 short sequences")
+
+
 @pytest.mark.parametrize("name", ["v2lite", "v3", "multitoken", "skewed"])
 def test_full_size_workloads_sampled_parity(name):
     wl = W.workload(name)
