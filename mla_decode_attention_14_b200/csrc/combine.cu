@@ -9,12 +9,76 @@
 // out = 0, lse = -inf. Sequences with no tokens at all (no piece) are written here too.
 //
 // One warp per (sequence, row); each lane owns 16 of the 512 output dims (four float4),
-// so every partial row is read as one coalesced 2 KB segment.
+// so every partial row is read as one coalesced 2 KB segment. Sequences of up to four pieces
+// (nearly all) load everything in one go; longer ones walk their pieces.
 #include "common.cuh"
 
 namespace mla {
 
 constexpr int kCombineWarps = 8;
+constexpr int kFastPieces = 4;
+
+__device__ __forceinline__ void store_row(__nv_bfloat16 *orow, float *lrow, const float (&acc)[16], float L, int lane) {
+    uint4 packed[2];
+    uint32_t *pw = reinterpret_cast<uint32_t *>(packed);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        __nv_bfloat162 two = __floats2bfloat162_rn(acc[2 * k], acc[2 * k + 1]);
+        pw[k] = *reinterpret_cast<uint32_t *>(&two);
+    }
+    reinterpret_cast<uint4 *>(orow)[0] = packed[0];
+    reinterpret_cast<uint4 *>(orow)[1] = packed[1];
+    if (lane == 0) *lrow = L;
+}
+
+// Rows of sequences with 0..kFastPieces pieces: the pieces' lse and this lane's 16 dims of each
+// partial row are loaded at once, then merged from registers.
+__device__ __forceinline__ void combine_few(int ns, int s0, int rows, int r, int lane, __nv_bfloat16 *orow, float *lrow,
+                                            const float *__restrict__ o_part, const float *__restrict__ lse_part) {
+    float ls[kFastPieces];
+    float4 v[kFastPieces][4];
+#pragma unroll
+    for (int s = 0; s < kFastPieces; ++s) {
+        if (s < ns) {
+            const size_t slot = (size_t)(s0 + s) * rows + r;
+            ls[s] = lse_part[slot];
+            const float4 *src = reinterpret_cast<const float4 *>(o_part + slot * kDv + lane * 16);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[s][k] = src[k];
+        } else {
+            ls[s] = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[s][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    float m = ls[0];
+#pragma unroll
+    for (int s = 1; s < kFastPieces; ++s) m = fmaxf(m, ls[s]);
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    if (m == -INFINITY) {  // no piece, or no visible key in any piece
+        store_row(orow, lrow, acc, -INFINITY, lane);
+        return;
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int s = 0; s < kFastPieces; ++s) sum += expf(ls[s] - m);  // empty pieces: e^-inf = 0
+    const float L = m + logf(sum);
+#pragma unroll
+    for (int s = 0; s < kFastPieces; ++s) {
+        const float wgt = expf(ls[s] - L);
+        if (wgt == 0.f) continue;  // empty piece (its o is 0) or negligible weight
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            acc[4 * k + 0] += wgt * v[s][k].x;
+            acc[4 * k + 1] += wgt * v[s][k].y;
+            acc[4 * k + 2] += wgt * v[s][k].z;
+            acc[4 * k + 3] += wgt * v[s][k].w;
+        }
+    }
+    store_row(orow, lrow, acc, L, lane);
+}
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
 combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts, int s_q, int h_q,
@@ -35,6 +99,10 @@ combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts,
     const int t = r / h_q, h = r % h_q;
     __nv_bfloat16 *orow = out + ((size_t)b * rows + r) * kDv + lane * 16;
     float *lrow = lse + ((size_t)b * h_q + h) * s_q + t;
+    if (ns <= kFastPieces) {  // common case: every load issued before any arithmetic (one memory round trip)
+        combine_few(ns, s0, rows, r, lane, orow, lrow, o_part, lse_part);
+        return;
+    }
 
     float m = -INFINITY;
     for (int s = lane; s < ns; s += 32) m = fmaxf(m, lse_part[(size_t)(s0 + s) * rows + r]);
@@ -71,16 +139,7 @@ combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts,
             acc[4 * k + 3] += wgt * v.w;
         }
     }
-    uint4 packed[2];
-    uint32_t *pw = reinterpret_cast<uint32_t *>(packed);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        __nv_bfloat162 two = __floats2bfloat162_rn(acc[2 * k], acc[2 * k + 1]);
-        pw[k] = *reinterpret_cast<uint32_t *>(&two);
-    }
-    reinterpret_cast<uint4 *>(orow)[0] = packed[0];
-    reinterpret_cast<uint4 *>(orow)[1] = packed[1];
-    if (lane == 0) *lrow = L;
+    store_row(orow, lrow, acc, L, lane);
 }
 
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q,
