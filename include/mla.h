@@ -213,6 +213,17 @@ int mla_check_status(void *stream);
  * counter; used to report how many of the library's kernels a benchmark ran). */
 int64_t mla_launch_count(void);
 
+/*
+ * Test of the failure path of the kernels' bounded waits (the pages have no counterpart; it
+ * exists so that the timeout path can be exercised without a fault). Launches, on `stream`,
+ * one CTA that waits, with the decode kernel's own wait primitive, on an mbarrier that nothing
+ * completes, for at most `spin_cycles` SM clock cycles (1e5 .. 4e9). The wait then gives up and
+ * raises the timeout bit of the device error word, so the next mla_check_status returns
+ * MLA_ERR_TIMEOUT. Returns MLA_ERR_INVALID_ARG for a bound outside the range, MLA_ERR_UNSUPPORTED
+ * without an sm_100 device, MLA_ERR_CUDA if the launch fails, else MLA_OK. Allocates nothing.
+ */
+int mla_selftest_wait_timeout(int64_t spin_cycles, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # exported C symbols, in the order include/mla.h declares them
 EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
            "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_host",
-           "mla_decode_noalloc", "mla_check_status", "mla_launch_count")
+           "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_selftest_wait_timeout")
 
 
 class MLAError(RuntimeError):
@@ -89,6 +89,8 @@ def lib():
         L.mla_check_status.restype = I
         L.mla_launch_count.argtypes = []
         L.mla_launch_count.restype = I64
+        L.mla_selftest_wait_timeout.argtypes = [I64, P]
+        L.mla_selftest_wait_timeout.restype = I
         _lib = L
     return _lib
 
@@ -291,3 +293,9 @@ def check_status(stream=None) -> int:
 def launch_count() -> int:
     """Kernels launched through the library by this process so far."""
     return int(lib().mla_launch_count())
+
+
+def selftest_wait_timeout(spin_cycles: int, stream=None) -> None:
+    """Run the kernels' bounded-wait primitive on an mbarrier nothing completes (see
+    mla_selftest_wait_timeout): the next check_status() returns MLA_ERR_TIMEOUT."""
+    _check("mla_selftest_wait_timeout", lib().mla_selftest_wait_timeout(int(spin_cycles), _stream(stream)))

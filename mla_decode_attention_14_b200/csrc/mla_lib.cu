@@ -5,3 +5,4 @@
 #include "combine.cu"
 #include "decode_sm100.cu"
 #include "noalloc.cu"
+#include "selftest.cu"

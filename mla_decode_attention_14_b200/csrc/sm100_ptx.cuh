@@ -73,17 +73,22 @@ MLA_DEV bool mbar_sleep_test_cluster(uint64_t *bar, uint32_t parity) {
         : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs) : "memory");
     return ok != 0;
 }
-MLA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// Waits for phase `parity` of `bar` for at most `spin` cycles; gives up early when *abort is set.
+// On expiry it sets *abort (so that the CTA's other roles stop too) and returns false.
+MLA_DEV bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort, long long spin) {
     if (mbar_test(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_sleep_test(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kSpinCycles) {
+        if (clock64() - t0 > spin) {
             *abort = 1;
             return false;
         }
     }
+}
+MLA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_wait_for(bar, parity, abort, kSpinCycles);
 }
 MLA_DEV bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_test_cluster(bar, parity)) return true;

@@ -116,3 +116,8 @@ def test_noalloc_scratch_constant_matches_header():
     src = open(HEADER).read()
     m = re.search(r"#define MLA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", src)
     assert m and int(m.group(1)) << int(m.group(2)) == mla.NOALLOC_SCRATCH_BYTES
+
+
+def test_selftest_bound_is_checked_on_host(L):
+    assert L.mla_selftest_wait_timeout(10, None) == 1  # MLA_ERR_INVALID_ARG: bound below 1e5 cycles
+    assert L.mla_selftest_wait_timeout(5_000_000_000, None) == 1

@@ -151,3 +151,14 @@ def test_host_entry_point_matches_device_path():
     lh = torch.empty((3, 64, 2), dtype=torch.float32).pin_memory()
     dec(qh, kvh, bth, slh, inp["scale"], True, oh, lh)
     assert torch.equal(oh, out_d.cpu()) and torch.equal(lh, lse_d.cpu())
+
+
+def test_bounded_wait_times_out_and_the_context_survives():
+    """A pipeline wait that nothing completes gives up after its bound, the status reports
+    MLA_ERR_TIMEOUT once, and the next decode on the same context is correct."""
+    assert mla.check_status() == 0
+    mla.selftest_wait_timeout(20_000_000)  # ~10 ms of SM clock
+    assert mla.check_status() == 5  # MLA_ERR_TIMEOUT
+    assert mla.check_status() == 0  # read and cleared
+    wl = W.workload("tiny")
+    parity.full_parity(W.make_inputs(wl, seed=2, tail="nan"), what="after a timeout")
