@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -56,13 +57,22 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source with comments removed and whitespace runs collapsed (string literals in these
+    sources hold no comment markers), so that edits to comments do not change the hash."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the code (not the comments) of the library's CUDA sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_decode_attention_14_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update((name + "\n" + _code_only(f.read())).encode())
     return h.hexdigest()[:16]
 
 

@@ -59,7 +59,7 @@ using namespace sm100;
 
 namespace dec {
 constexpr int kStages = 5;
-constexpr int kFirstSoftWarp = 4;                 // warpgroup 0: TMA producer and the three MMA-issuing warps
+constexpr int kFirstSoftWarp = 4;                 // warpgroup 0: TMA producer, Gemm1 issuer, (idle), Gemm2 issuer
 constexpr int kSoftWarps = 8;                     // two per SM sub-partition
 constexpr int kThreads = 32 * (kFirstSoftWarp + kSoftWarps);  // 384
 constexpr int kTq = 2;                            // token halves per block
@@ -89,7 +89,7 @@ constexpr int kXchgOffBytes = 2 * kTq * 128 * 4;   // two slots of 128 rows x 2 
 
 struct __align__(1024) Smem {
     uint8_t stage[kStages][kStageBytes];  // KV ring
-    uint4 xchg[(kXchgEBytes + kXchgOffBytes) / 16];  // peer E factors (fp16) [slot][token half][16 B][row]
+    uint4 xchg[(kXchgEBytes + kXchgOffBytes) / 16];  // peer factors R (fp16) [slot][token half][16 B][row]
                                                      // + row offsets (fp32) [slot][token half][row]
     float xmax[2][kTq][128];  // per-row exchange between the two token halves (block max bound; sums)
     uint8_t q_rope[128 * 64];             // rotary query dims [128 rows x 32], K-major, 64-byte swizzle
@@ -365,7 +365,7 @@ __device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int 
     return true;
 }
 
-// E (fp16) and m (fp32) of block g into the peer CTA's receive slot g % 2 (the first block of a
+// R (fp16) and m (fp32) of block g into the peer CTA's receive slot g % 2 (the first block of a
 // part; later blocks are sent from the softmax loop as their exponentials are computed).
 __device__ __forceinline__ void send_factors(const SoftCtx &c, int g, const float (&e)[kTokPer], float m_own) {
     if (!c.warp_ok) return;
@@ -426,7 +426,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     c.xfull_peer0 = map_to_rank(&sm.xfull[0], peer);
     const uint32_t xchg_peer = c.xchg_peer, xfull_peer0 = c.xfull_peer0;
     const int nvalid_warps = min(4, (p.rows - group * 128 + 31) / 32);
-    const uint32_t xbytes = (uint32_t)nvalid_warps * kTq * 32 * (2 * kTokPer + 4);  // E (fp16) + offset
+    const uint32_t xbytes = (uint32_t)nvalid_warps * kTq * 32 * (2 * kTokPer + 4);  // R (fp16) + offset
     const int t_q = c.row_ok ? c.r / p.h_q : 0, h_idx = c.row_ok ? c.r % p.h_q : 0;
     const float sl2 = p.scale_log2;
     volatile int *abort = &sm.abort;
