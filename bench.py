@@ -249,6 +249,9 @@ def main():
     ap.add_argument("--workload", default="v3", choices=W.NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--graph-steps", type=int, default=-1,
+                    help="replays of the step captured in a CUDA graph, reported under 'graph' "
+                         "(default: as many as --steps; 0: skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--max-batch", type=int, default=0,
                     help="keep only the first N sequences (for profiler captures of a smaller slice)")
@@ -352,6 +355,37 @@ def main():
     value = job_throughput(counts["bytes"], world, ms_per_step)
     tflops = counts["flops"] * world / (ms_per_step * 1e-3) / 1e12
 
+    # the same step captured once in a CUDA graph and replayed (launch overhead removed); reported
+    # beside the eager numbers, which stay the headline (they are the library's own launches)
+    graph_ms = None
+    graph_steps = args.steps if args.graph_steps < 0 else args.graph_steps
+    if flush is None and graph_steps > 0:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        g0.record(stream)
+        for _ in range(graph_steps):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks([g0.elapsed_time(g1) / graph_steps], dev)[0]
+        del graph
+        st = mla.check_status()
+        if st != 0:
+            raise SystemExit("device error status %d in the graph replays" % st)
+
     # end to end through the host entry point: pinned host inputs in, host outputs out
     e2e = None
     if args.e2e_steps > 0:
@@ -407,7 +441,10 @@ def main():
                                   if flush is None else "inputs (%.1f MB) fit in L2: a 256 MB write flushes L2 between "
                                   "steps, outside the timed steps" % (in_bytes / 1e6)),
                            "parallelism": "independent batch per GPU" if world > 1 else "1 GPU"},
-                "roofline": roof, "clocks": clk.summary(), "e2e": e2e, "gpu_launches": launches}
+                "roofline": roof, "clocks": clk.summary(), "e2e": e2e, "gpu_launches": launches,
+                "graph": None if graph_ms is None else {
+                    "ms_per_step": graph_ms, "value": job_throughput(counts["bytes"], world, graph_ms), "unit": "TB/s",
+                    "note": "the same step (metadata + split + combine) captured once in a CUDA graph and replayed"}}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, inp)
         print(json.dumps(line), flush=True)
