@@ -15,6 +15,11 @@ Recipe (the same for every workload):
     parity runs (they must not influence the result) or N(0, 1) for timing runs;
   * scale = 192 ** -0.5 for every workload.
 
+fp8 cache (``make_inputs_fp8``): the same q, block table and tails; per token a 640-byte
+record of 512 latent dims as OCP E4M3 bytes -- N(0, 1) float32 divided by the latent
+scale (default 2^-6), clipped to +-448 and rounded to E4M3 (nearest, ties to even, by
+torch's float8_e4m3fn cast) -- followed by the 64 rotary dims as bf16 N(0, 1).
+
 Workloads (sizes as named by the library's benchmark list):
   tiny        b=2,   h_q=16,  s_q=1, seqlens {100, 257}
   v2lite      b=64,  h_q=16,  s_q=1, every seqlen 4096      (DeepSeek-V2-Lite head count)
@@ -35,6 +40,9 @@ D_V = 512
 BLK = 64
 SCALE = 192.0 ** -0.5
 BF16_NAN = 0x7FC0
+F8_REC = 640            # fp8 cache: bytes per token (512 E4M3 latent + 64 bf16 rotary)
+F8_NAN = 0x7F           # an E4M3 NaN
+F8_SCALE = 2.0 ** -6    # default latent scale of the synthetic fp8 cache
 
 
 @dataclass
@@ -155,14 +163,56 @@ def make_inputs(wl: Workload, seed: int = 0, tail: str = "nan", spare_blocks: in
             "scale": wl.scale, "causal": wl.causal, "num_blocks": nblk}
 
 
-def algorithmic_counts(wl: Workload):
+def _e4m3_codes(x: np.ndarray) -> np.ndarray:
+    import torch
+    t = torch.from_numpy(np.clip(x, -448.0, 448.0).astype(np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def make_inputs_fp8(wl: Workload, seed: int = 0, tail: str = "nan", spare_blocks: int = 0,
+                    kv_scale: float = F8_SCALE, chunk_tokens: int = 1 << 16):
+    """Draw q, an fp8 paged cache and the block table for ``wl``.
+
+    Returns a dict with ``q`` uint16 [b, s_q, h_q, 576] (bf16 bits), ``kv8`` uint8
+    [num_blocks, 64, 1, 640] (per token 512 E4M3 bytes then 64 bf16 little-endian),
+    ``kv_scale`` (a latent byte x stands for kv_scale * e4m3(x)), ``block_table``,
+    ``seqlens``, ``scale``, ``causal``, ``num_blocks``.
+    """
+    rng = np.random.default_rng([seed, 3])
+    bt, nblk = block_layout(wl.seqlens, rng, spare_blocks)
+    q = _normal_bf16(rng, (wl.batch, wl.s_q, wl.h_q, D_QK))
+    ntok = max(nblk, 1) * BLK
+    kv8 = np.empty((ntok, F8_REC), dtype=np.uint8)
+    for lo in range(0, ntok, chunk_tokens):
+        hi = min(ntok, lo + chunk_tokens)
+        lat = rng.standard_normal((hi - lo, D_V), dtype=np.float32) / np.float32(kv_scale)
+        kv8[lo:hi, :D_V] = _e4m3_codes(lat)
+        rope = f32_to_bf16_bits(rng.standard_normal((hi - lo, D_QK - D_V), dtype=np.float32))
+        kv8[lo:hi, D_V:] = np.ascontiguousarray(rope.astype("<u2")).view(np.uint8).reshape(hi - lo, -1)
+    kv8 = kv8.reshape(max(nblk, 1), BLK, 1, F8_REC)
+    if tail == "nan":
+        nan_rope = np.frombuffer(np.array([BF16_NAN], dtype="<u2").tobytes() * (D_QK - D_V), dtype=np.uint8)
+        for i, n in enumerate(wl.seqlens):
+            n = int(n)
+            w = (max(n, 0) + BLK - 1) // BLK
+            if w > 0 and n % BLK:
+                blk = kv8[bt[i, w - 1], n % BLK:, 0, :]
+                blk[:, :D_V] = F8_NAN
+                blk[:, D_V:] = nan_rope
+    elif tail != "normal":
+        raise ValueError(tail)
+    return {"q": q, "kv8": kv8, "kv_scale": float(kv_scale), "block_table": bt, "seqlens": wl.seqlens.copy(),
+            "scale": wl.scale, "causal": wl.causal, "num_blocks": nblk}
+
+
+def algorithmic_counts(wl: Workload, kv: str = "bf16"):
     """Algorithmic bytes and flops of one decode of ``wl``.
 
-    bytes = 1152 per KV token (576 bf16, keys and values share the vector) plus 1152 per
-    query row; flops = 2 * (576 + 512) per (visible key, query row).
+    bytes = 1152 per KV token (576 bf16, keys and values share the vector; 640 for the
+    fp8 cache) plus 1152 per query row; flops = 2 * (576 + 512) per (visible key, query row).
     """
     n = np.maximum(wl.seqlens.astype(np.int64), 0)
-    kv_bytes = int(n.sum()) * D_QK * 2
+    kv_bytes = int(n.sum()) * (F8_REC if kv == "fp8" else D_QK * 2)
     q_bytes = wl.batch * wl.rows * D_QK * 2
     vis = 0
     for t in range(wl.s_q):

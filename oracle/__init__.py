@@ -28,6 +28,7 @@ _lib = None
 D_QK = 576
 D_V = 512
 BLK = 64
+F8_REC = 640  # fp8 cache: bytes per token
 
 
 def build(force: bool = False) -> str:
@@ -53,6 +54,12 @@ def _load():
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                       ctypes.c_int, P, P, P, ctypes.c_int64, ctypes.c_int]
         lib.oracle_decode.restype = ctypes.c_int
+        lib.oracle_decode_fp8.argtypes = [P, P, ctypes.c_double, ctypes.c_int64, P, ctypes.c_int64, P,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                          ctypes.c_int, P, P, P, ctypes.c_int64, ctypes.c_int]
+        lib.oracle_decode_fp8.restype = ctypes.c_int
+        lib.oracle_e4m3_decode.argtypes = [P, ctypes.c_int64, P]
+        lib.oracle_e4m3_decode.restype = None
         _lib = lib
     return _lib
 
@@ -110,3 +117,42 @@ def decode(q_bits, kv_bits, block_table, seqlens, scale: float, causal: bool,
     if rc != 0:
         raise ValueError("oracle_decode failed (rc=%d)" % rc)
     return out, lse
+
+
+def decode_fp8(q_bits, kv8, kv_scale: float, block_table, seqlens, scale: float, causal: bool,
+               tasks=None, nthreads: int | None = None):
+    """Exact (double) MLA decode attention over the fp8 cache.
+
+    ``kv8``: uint8 ``[num_blocks, 64, 1, 640]`` (or ``[num_blocks, 64, 640]``): per token
+    512 OCP E4M3 latent bytes, each standing for ``kv_scale * e4m3(byte)``, then the 64
+    rotary dims as little-endian bf16. Everything else as :func:`decode`.
+    """
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kv = np.ascontiguousarray(kv8, dtype=np.uint8)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    b, s_q, h_q, d = q.shape
+    assert d == D_QK and kv.shape[-1] == F8_REC and kv.shape[1] == BLK
+    out = np.full((b, s_q, h_q, D_V), np.nan, dtype=np.float64)
+    lse = np.full((b, h_q, s_q), np.nan, dtype=np.float64)
+    if tasks is not None:
+        tk = np.ascontiguousarray(tasks, dtype=np.int32).reshape(-1, 3)
+        tptr, nt = _ptr(tk), tk.shape[0]
+    else:
+        tk, tptr, nt = None, None, 0
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().oracle_decode_fp8(_ptr(q), _ptr(kv), float(kv_scale), kv.shape[0], _ptr(bt),
+                                   bt.shape[1] if bt.ndim == 2 else 0, _ptr(sl), b, s_q, h_q, float(scale),
+                                   int(bool(causal)), _ptr(out), _ptr(lse), tptr, nt, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_decode_fp8 failed (rc=%d)" % rc)
+    return out, lse
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """OCP E4M3 bytes -> float64, as the oracle reads the fp8 cache."""
+    x = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(x.shape, dtype=np.float64)
+    _load().oracle_e4m3_decode(_ptr(x), x.size, _ptr(out))
+    return out

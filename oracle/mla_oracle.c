@@ -25,6 +25,11 @@
  * Precision: every product and sum is taken in double from exactly up-converted
  * bf16 inputs; the outputs are doubles (never rounded to bf16 here).
  *
+ * The fp8 cache (oracle_decode_fp8) holds, per token, 512 latent dims as OCP E4M3 bytes
+ * and the 64 rotary dims as bf16; a latent byte x stands for kv_scale * e4m3(x). Keys
+ * and values are those dequantized vectors; everything after that is the same
+ * attention, in double.
+ *
  * Parity pins (see tests/test_oracle*.py): dense non-paged brute force through a
  * library softmax-attention routine, single-token sequences, block-permutation
  * invariance, lse against a library log-sum-exp, q = 0 closed form, NaN-poisoned
@@ -47,6 +52,23 @@ static double bf16_bits_to_double(uint16_t h) {
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* OCP 8-bit floating point (OFP8), format E4M3, exactly: bit 7 sign, bits 6..3
+ * exponent field E (bias 7), bits 2..0 mantissa M. E = 0: (M / 8) * 2^-6
+ * (subnormal; M = 0 is a signed zero). E = 15 and M = 7: NaN. Otherwise
+ * (1 + M / 8) * 2^(E - 7); the largest finite magnitude is 1.75 * 2^8 = 448. There
+ * are no infinities. */
+static double e4m3_to_double(uint8_t x) {
+    const int sign = x >> 7, e = (x >> 3) & 15, m = x & 7;
+    double v;
+    if (e == 15 && m == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
 }
 
 /* ------------------------------------------------------------------------- */
@@ -143,8 +165,12 @@ int oracle_metadata(const int32_t *seqlens, int batch, int num_parts, int fixed_
 /* Only the first ceil(V/64) block-table entries of a row are read; the other */
 /* entries and the cache rows past V are never touched.                        */
 /* ------------------------------------------------------------------------- */
+#define OR_F8_REC 640 /* fp8 cache: bytes per token (512 E4M3 + 64 bf16) */
+
 typedef struct {
     const uint16_t *q, *kv;
+    const uint8_t *kv8; /* fp8 cache (kv == NULL), with its latent scale */
+    double kv_scale;
     int64_t num_blocks;
     const int32_t *block_table;
     int64_t bt_stride;
@@ -158,6 +184,21 @@ typedef struct {
     pthread_mutex_t lock;
     int error;
 } dec_job;
+
+/* The 576 dims of cache row `row` (physical block * 64 + slot) as doubles. */
+static void load_key(const dec_job *J, int64_t row, double *k) {
+    if (J->kv) {
+        const uint16_t *src = J->kv + (size_t)row * OR_D_QK;
+        for (int d = 0; d < OR_D_QK; ++d) k[d] = bf16_bits_to_double(src[d]);
+    } else {
+        const uint8_t *src = J->kv8 + (size_t)row * OR_F8_REC;
+        for (int d = 0; d < OR_D_V; ++d) k[d] = J->kv_scale * e4m3_to_double(src[d]);
+        for (int d = OR_D_V; d < OR_D_QK; ++d) {
+            const uint8_t *r = src + OR_D_V + 2 * (d - OR_D_V); /* little-endian bf16 */
+            k[d] = bf16_bits_to_double((uint16_t)(r[0] | (r[1] << 8)));
+        }
+    }
+}
 
 static int one_row(dec_job *J, int b, int t, int h, double *scores, double *acc) {
     const int rows = J->s_q * J->h_q;
@@ -181,13 +222,13 @@ static int one_row(dec_job *J, int b, int t, int h, double *scores, double *acc)
     double qd[OR_D_QK];
     for (int d = 0; d < OR_D_QK; ++d) qd[d] = bf16_bits_to_double(qrow[d]);
 
-    double m = -INFINITY;
+    double m = -INFINITY, key[OR_D_QK];
     for (int64_t j = 0; j < V; ++j) {
         int32_t phys = J->block_table[(size_t)b * J->bt_stride + j / OR_BLK];
         if (phys < 0 || phys >= J->num_blocks) return -1;
-        const uint16_t *key = J->kv + ((size_t)phys * OR_BLK + (size_t)(j % OR_BLK)) * OR_D_QK;
+        load_key(J, (int64_t)phys * OR_BLK + j % OR_BLK, key);
         double dot = 0.0;
-        for (int d = 0; d < OR_D_QK; ++d) dot += qd[d] * bf16_bits_to_double(key[d]);
+        for (int d = 0; d < OR_D_QK; ++d) dot += qd[d] * key[d];
         scores[j] = J->scale * dot;
         if (scores[j] > m) m = scores[j];
     }
@@ -197,9 +238,9 @@ static int one_row(dec_job *J, int b, int t, int h, double *scores, double *acc)
     for (int d = 0; d < OR_D_V; ++d) acc[d] = 0.0;
     for (int64_t j = 0; j < V; ++j) {
         int32_t phys = J->block_table[(size_t)b * J->bt_stride + j / OR_BLK];
-        const uint16_t *val = J->kv + ((size_t)phys * OR_BLK + (size_t)(j % OR_BLK)) * OR_D_QK;
+        load_key(J, (int64_t)phys * OR_BLK + j % OR_BLK, key); /* the value is its first 512 dims */
         double p = exp(scores[j] - L);
-        for (int d = 0; d < OR_D_V; ++d) acc[d] += p * bf16_bits_to_double(val[d]);
+        for (int d = 0; d < OR_D_V; ++d) acc[d] += p * key[d];
     }
     for (int d = 0; d < OR_D_V; ++d) o[d] = acc[d];
     *lse = L;
@@ -262,11 +303,11 @@ static void *dec_worker(void *arg) {
  * Returns 0; -1 bad arguments; -2 out of memory; -3 a block-table entry that must be
  * read is outside [0, num_blocks).
  */
-int oracle_decode(const uint16_t *q, const uint16_t *kv_cache, int64_t num_blocks,
-                  const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
-                  int batch, int s_q, int h_q, double scale, int causal, double *out,
-                  double *lse, const int32_t *tasks, int64_t ntasks, int nthreads) {
-    if (!q || !kv_cache || !block_table || !seqlens || !out || !lse) return -1;
+static int run_decode(const uint16_t *q, const uint16_t *kv_cache, const uint8_t *kv8, double kv_scale,
+                      int64_t num_blocks, const int32_t *block_table, int64_t bt_stride,
+                      const int32_t *seqlens, int batch, int s_q, int h_q, double scale, int causal,
+                      double *out, double *lse, const int32_t *tasks, int64_t ntasks, int nthreads) {
+    if (!q || (!kv_cache && !kv8) || !block_table || !seqlens || !out || !lse) return -1;
     if (batch < 0 || s_q < 1 || h_q < 1 || nthreads < 1 || num_blocks < 0) return -1;
     if (tasks && ntasks < 0) return -1;
     for (int b = 0; b < batch; ++b) {
@@ -275,7 +316,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *kv_cache, int64_t num_block
     }
     dec_job J;
     memset(&J, 0, sizeof J);
-    J.q = q; J.kv = kv_cache; J.num_blocks = num_blocks; J.block_table = block_table;
+    J.q = q; J.kv = kv_cache; J.kv8 = kv8; J.kv_scale = kv_scale; J.num_blocks = num_blocks; J.block_table = block_table;
     J.bt_stride = bt_stride; J.seqlens = seqlens; J.batch = batch; J.s_q = s_q;
     J.h_q = h_q; J.causal = causal; J.scale = scale; J.out = out; J.lse = lse;
     J.tasks = tasks; J.ntasks = ntasks; J.next = 0; J.error = 0;
@@ -292,4 +333,32 @@ int oracle_decode(const uint16_t *q, const uint16_t *kv_cache, int64_t num_block
     free(th);
     pthread_mutex_destroy(&J.lock);
     return J.error;
+}
+
+int oracle_decode(const uint16_t *q, const uint16_t *kv_cache, int64_t num_blocks,
+                  const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                  int batch, int s_q, int h_q, double scale, int causal, double *out,
+                  double *lse, const int32_t *tasks, int64_t ntasks, int nthreads) {
+    if (!kv_cache) return -1;
+    return run_decode(q, kv_cache, NULL, 0.0, num_blocks, block_table, bt_stride, seqlens, batch, s_q,
+                      h_q, scale, causal, out, lse, tasks, ntasks, nthreads);
+}
+
+/*
+ * The same attention over the fp8 cache: kv8 is uint8[num_blocks, 64, 640], per token
+ * 512 E4M3 latent bytes (value kv_scale * e4m3(byte)) then 64 bf16 rotary dims
+ * (little-endian). Arguments and return codes as oracle_decode.
+ */
+int oracle_decode_fp8(const uint16_t *q, const uint8_t *kv8, double kv_scale, int64_t num_blocks,
+                      const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                      int batch, int s_q, int h_q, double scale, int causal, double *out,
+                      double *lse, const int32_t *tasks, int64_t ntasks, int nthreads) {
+    if (!kv8) return -1;
+    return run_decode(q, NULL, kv8, kv_scale, num_blocks, block_table, bt_stride, seqlens, batch, s_q,
+                      h_q, scale, causal, out, lse, tasks, ntasks, nthreads);
+}
+
+/* E4M3 byte -> double, for the tests that pin the decoding itself. */
+void oracle_e4m3_decode(const uint8_t *x, int64_t n, double *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_double(x[i]);
 }
