@@ -121,7 +121,8 @@ int mla_get_metadata(const int32_t *seqlens, int batch, int h_q, int s_q, int nu
  *                are read; others may hold anything (e.g. -1)
  *   seqlens      int32[batch]                     tokens in each sequence (<= 64*bt_stride)
  *   tile_meta, num_splits, num_parts, as produced by mla_get_metadata for these seqlens
- *   scale        multiplies q.k before the softmax (finite)
+ *   scale        multiplies q.k before the softmax (finite, >= 0: the kernel takes the row
+ *                maximum of the raw scores and scales it afterwards)
  *   causal       0/1, masking between the s_q query tokens (see top of file)
  *   out          bf16[batch, s_q, h_q, 512]       written (round to nearest even)
  *   lse          fp32[batch, h_q, s_q]            written (natural log; -inf if no key)

@@ -140,7 +140,7 @@ int validate_decode(const void *q, const void *kv, int64_t num_blocks, const int
     if (num_parts < 1 || num_parts > 65535) return MLA_ERR_INVALID_ARG;
     if (num_blocks < 1 || num_blocks > (int64_t)(INT32_MAX / MLA_BLOCK_TOKENS)) return MLA_ERR_INVALID_ARG;
     if (bt_stride < 1 || bt_stride > (int64_t)INT32_MAX) return MLA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale >= 0.f)) return MLA_ERR_INVALID_ARG;  // the max commutes with scale >= 0
     if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
         !aligned(ws, 256) || !aligned(bt, 4) || !aligned(seqlens, 4) || !aligned(tile_meta, 4) ||

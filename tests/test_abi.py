@@ -71,7 +71,7 @@ def _decode_call(L, **kw):
 @pytest.mark.parametrize("bad", [
     dict(q=None), dict(kv=None), dict(out=None), dict(ws=None), dict(q=FAKE + 8), dict(kv=FAKE + 2),
     dict(ws=FAKE + 16), dict(b=0), dict(s_q=0), dict(h_q=0), dict(h_q=1025), dict(P=0), dict(nblk=0),
-    dict(bts=0), dict(scale=float("nan")), dict(scale=float("inf")), dict(causal=2),
+    dict(bts=0), dict(scale=float("nan")), dict(scale=float("inf")), dict(scale=-0.1), dict(causal=2),
 ])
 def test_invalid_arguments_rejected_on_host(L, bad):
     assert _decode_call(L, **bad) == 1  # MLA_ERR_INVALID_ARG
