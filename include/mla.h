@@ -62,6 +62,7 @@ extern "C" {
 #define MLA_TILE_META_INTS 8  /* int32 per part in tile_meta                   */
 #define MLA_MAX_ROWS 1024     /* max s_q * h_q per call                        */
 #define MLA_MAX_BATCH 65536   /* max batch per call                            */
+#define MLA_FP8_RECORD_BYTES 640 /* fp8 cache: bytes per token (512 E4M3 + 64 bf16) */
 
 typedef enum mla_status {
     MLA_OK = 0,
@@ -70,7 +71,9 @@ typedef enum mla_status {
     MLA_ERR_WORKSPACE = 3,   /* workspace smaller than mla_workspace_bytes()      */
     MLA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                 */
     MLA_ERR_TIMEOUT = 5,     /* a device pipeline wait hit its bound (reported by mla_check_status) */
-    MLA_ERR_BOUNDS = 6       /* a block-table entry outside [0, num_blocks) was needed */
+    MLA_ERR_BOUNDS = 6,      /* a block-table entry outside [0, num_blocks) was needed */
+    MLA_ERR_RANGE = 7        /* fp8 cache: a query value outside the range of its fp16 form
+                                (reported by mla_check_status) */
 } mla_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -148,6 +151,39 @@ int mla_decode_split(const void *q, const void *kv_cache, int64_t num_blocks,
 int mla_decode_combine(const int32_t *num_splits, int num_parts, int batch, int s_q, int h_q,
                        void *out, float *lse, const void *workspace, size_t workspace_bytes,
                        void *stream);
+
+/*
+ * The same decode over an FP8 latent cache. The pages name FP8 precision as a tuning option for
+ * more throughput ("Playing DeepSeek on the cloud, part 5: ... FlashMLA accelerating
+ * DeepSeek-V2-Lite inference", section 4 "developer practice", item 2 "monitoring and tuning"),
+ * and FP8 as the data type DeepEP dispatches natively ("Deep analysis of the DeepSeek Infra
+ * open-source releases", DAY2 DeepEP, project feature 3); neither fixes a cache format, so this
+ * one is the library's own:
+ *   kv_cache_fp8  uint8[num_blocks, 64, 1, MLA_FP8_RECORD_BYTES], 16-byte aligned; per token
+ *                 bytes [0, 512) are the 512 latent dims as OCP E4M3 (1 sign, 4 exponent bits
+ *                 with bias 7, 3 mantissa bits; no infinities), and bytes [512, 640) are the 64
+ *                 rotary dims as little-endian bf16
+ *   kv_scale      latent byte x stands for kv_scale * e4m3(x) (one scale for the whole cache;
+ *                 finite, in [2^-64, 2^64]); the rotary dims are not scaled
+ * Keys are the dequantized 576-d vectors and values their first 512 dims; all other arguments,
+ * outputs, the workspace and the two-kernel split are as for mla_decode.
+ * How it computes: the latent query dims are multiplied by kv_scale / 2^floor(log2 kv_scale) and
+ * rounded to fp16 (a relative error of at most 2^-11 per element; every E4M3 value is an fp16
+ * number, so the cache side is exact), the products and sums are fp32, the probabilities P are
+ * rounded to fp16 for P.V. A query value that does not fit fp16 after that multiplication (or is
+ * not finite) sets MLA_ERR_RANGE, which mla_check_status reports; the results are then undefined.
+ */
+int mla_decode_fp8(const void *q, const void *kv_cache_fp8, int64_t num_blocks, float kv_scale,
+                   const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                   const int32_t *tile_meta, const int32_t *num_splits, int num_parts, int batch,
+                   int s_q, int h_q, float scale, int causal, void *out, float *lse, void *workspace,
+                   size_t workspace_bytes, void *stream);
+/* The split kernel alone (mla_decode_combine finishes, as for mla_decode_split). */
+int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_blocks, float kv_scale,
+                         const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                         const int32_t *tile_meta, const int32_t *num_splits, int num_parts,
+                         int batch, int s_q, int h_q, float scale, int causal, void *out,
+                         float *lse, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * End-to-end call on HOST buffers: copies the inputs host->device, runs metadata +

@@ -25,6 +25,7 @@ import torch
 D_QK = 576
 D_V = 512
 BLOCK = 64
+FP8_RECORD_BYTES = 640  # MLA_FP8_RECORD_BYTES in include/mla.h
 META_INTS = 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,11 +34,13 @@ _lib = None
 
 MLA_OK = 0
 STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_WORKSPACE",
-                4: "MLA_ERR_CUDA", 5: "MLA_ERR_TIMEOUT", 6: "MLA_ERR_BOUNDS"}
+                4: "MLA_ERR_CUDA", 5: "MLA_ERR_TIMEOUT", 6: "MLA_ERR_BOUNDS",
+                7: "MLA_ERR_RANGE"}
 
 # exported C symbols, in the order include/mla.h declares them
 EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
-           "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_host",
+           "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_fp8",
+           "mla_decode_split_fp8", "mla_decode_host",
            "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_selftest_wait_timeout")
 
 
@@ -77,6 +80,10 @@ def lib():
         dec = [P, P, I64, P, I64, P, P, P, I, I, I, I, F, I, P, P, P, SZ, P]
         for name in ("mla_decode", "mla_decode_split"):
             getattr(L, name).argtypes = dec
+            getattr(L, name).restype = I
+        dec8 = dec[:3] + [F] + dec[3:]  # kv_scale after num_blocks
+        for name in ("mla_decode_fp8", "mla_decode_split_fp8"):
+            getattr(L, name).argtypes = dec8
             getattr(L, name).restype = I
         L.mla_decode_noalloc.argtypes = dec[:16] + [P]
         L.mla_decode_noalloc.restype = I
@@ -163,22 +170,75 @@ def get_metadata(seqlens: torch.Tensor, h_q: int, s_q: int, num_parts: int | Non
 
 def _decode_args(q, kv_cache, block_table, seqlens, meta):
     _need(q, "q", torch.bfloat16, 4)
-    _need(kv_cache, "kv_cache", torch.bfloat16)
     _need(block_table, "block_table", torch.int32, 2)
     _need(seqlens, "seqlens", torch.int32, 1)
     b, s_q, h_q, d = q.shape
     if d != D_QK:
         raise ValueError("q last dim must be %d" % D_QK)
-    if kv_cache.dim() == 4:
-        if kv_cache.shape[1:] != (BLOCK, 1, D_QK):
+    if kv_cache is not None:  # bf16 cache (the fp8 one is checked by decode_fp8)
+        _need(kv_cache, "kv_cache", torch.bfloat16)
+        if kv_cache.dim() == 4:
+            if kv_cache.shape[1:] != (BLOCK, 1, D_QK):
+                raise ValueError("kv_cache must be [num_blocks, 64, 1, 576], got %s" % (tuple(kv_cache.shape),))
+        elif kv_cache.dim() != 3 or kv_cache.shape[1:] != (BLOCK, D_QK):
             raise ValueError("kv_cache must be [num_blocks, 64, 1, 576], got %s" % (tuple(kv_cache.shape),))
-    elif kv_cache.dim() != 3 or kv_cache.shape[1:] != (BLOCK, D_QK):
-        raise ValueError("kv_cache must be [num_blocks, 64, 1, 576], got %s" % (tuple(kv_cache.shape),))
     if block_table.shape[0] != b or seqlens.shape[0] != b:
         raise ValueError("batch mismatch between q, block_table and seqlens")
     if meta.h_q != h_q or meta.s_q != s_q or meta.num_splits.shape[0] != b + 1:
         raise ValueError("metadata was computed for another shape")
     return b, s_q, h_q
+
+
+def _outputs(b, s_q, h_q, meta, dev, out, lse, workspace):
+    if out is None:
+        out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    ws_bytes = workspace_bytes(b, s_q, h_q, meta.num_parts)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    if workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError("workspace too small: need %d bytes" % ws_bytes)
+    return out, lse, workspace, ws_bytes
+
+
+def decode_fp8(q: torch.Tensor, kv_cache_fp8: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+               scale: float, kv_scale: float, causal: bool, meta: Metadata, out: torch.Tensor | None = None,
+               lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None,
+               phase: str = "both"):
+    """MLA decode attention over an fp8 cache (``mla_decode_fp8``).
+
+    ``kv_cache_fp8``: uint8 ``[num_blocks, 64, 1, 640]`` (or ``[num_blocks, 64, 640]``), per
+    token 512 E4M3 latent bytes standing for ``kv_scale * e4m3(byte)``, then 64 bf16 rotary
+    dims. Returns ``(out, lse)`` as :func:`decode`; ``phase`` as there.
+    """
+    kv = kv_cache_fp8
+    _need(kv, "kv_cache_fp8", torch.uint8)
+    if not ((kv.dim() == 4 and kv.shape[1:] == (BLOCK, 1, FP8_RECORD_BYTES)) or
+            (kv.dim() == 3 and kv.shape[1:] == (BLOCK, FP8_RECORD_BYTES))):
+        raise ValueError("kv_cache_fp8 must be uint8 [num_blocks, 64, 1, %d], got %s"
+                         % (FP8_RECORD_BYTES, tuple(kv.shape)))
+    b, s_q, h_q = _decode_args(q, None, block_table, seqlens, meta)
+    out, lse, workspace, ws_bytes = _outputs(b, s_q, h_q, meta, q.device, out, lse, workspace)
+    st = _stream(stream)
+    L = lib()
+    with torch.cuda.device(q.device):
+        if phase in ("both", "split"):
+            fn = L.mla_decode_fp8 if phase == "both" else L.mla_decode_split_fp8
+            _check("mla_decode_fp8", fn(q.data_ptr(), kv.data_ptr(), kv.shape[0], float(kv_scale),
+                                        block_table.data_ptr(), block_table.shape[1], seqlens.data_ptr(),
+                                        meta.tile_meta.data_ptr(), meta.num_splits.data_ptr(), meta.num_parts, b,
+                                        s_q, h_q, float(scale), int(bool(causal)), out.data_ptr(), lse.data_ptr(),
+                                        workspace.data_ptr(), ws_bytes, st))
+        elif phase == "combine":
+            _check("mla_decode_combine", L.mla_decode_combine(meta.num_splits.data_ptr(), meta.num_parts, b, s_q,
+                                                              h_q, out.data_ptr(), lse.data_ptr(),
+                                                              workspace.data_ptr(), ws_bytes, st))
+        else:
+            raise ValueError(phase)
+    return out, lse
 
 
 def decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,

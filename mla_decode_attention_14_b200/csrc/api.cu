@@ -19,7 +19,7 @@ cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, 
                            __nv_bfloat16 *out, float *lse, const float *o_part,
                            const float *lse_part, cudaStream_t stream);
 cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
-                                cudaStream_t stream);
+                                bool fp8, cudaStream_t stream);
 
 static std::atomic<int64_t> g_launches{0};
 
@@ -50,6 +50,9 @@ int check_device() {
 // ---- TMA descriptors of the paged cache, viewed as a 2-D bf16 tensor [num_blocks * 64, 576]:
 // "latent" boxes are 64 tokens x 64 dims with the 128-byte swizzle, "rope" boxes are
 // 64 tokens x 32 dims with the 64-byte swizzle (the layouts the MMA descriptors expect).
+// fp8 cache ([num_blocks * 64] records of 640 bytes): "latent" boxes are 64 tokens x 128 bytes
+// (E4M3) with the 128-byte swizzle over a uint8 view, "rope" boxes 64 tokens x 32 bf16 with the
+// 64-byte swizzle over a [rows, 320] bf16 view of the same records.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -70,7 +73,7 @@ EncodeTiledFn encode_fn() {
 struct MapEntry {
     const void *kv;
     int64_t num_blocks;
-    int device;
+    int device, fp8;
     CUtensorMap lat, rope;
 };
 constexpr int kMapCache = 16;
@@ -78,12 +81,13 @@ MapEntry g_maps[kMapCache];
 int g_maps_used = 0, g_maps_next = 0;
 std::mutex g_maps_mu;
 
-int cache_maps(const void *kv, int64_t num_blocks, CUtensorMap *lat, CUtensorMap *rope) {
+int cache_maps(const void *kv, int64_t num_blocks, int fp8, CUtensorMap *lat, CUtensorMap *rope) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_maps_mu);
     for (int k = 0; k < g_maps_used; ++k) {
-        if (g_maps[k].kv == kv && g_maps[k].num_blocks == num_blocks && g_maps[k].device == dev) {
+        if (g_maps[k].kv == kv && g_maps[k].num_blocks == num_blocks && g_maps[k].device == dev &&
+            g_maps[k].fp8 == fp8) {
             *lat = g_maps[k].lat;
             *rope = g_maps[k].rope;
             return MLA_OK;
@@ -95,11 +99,16 @@ int cache_maps(const void *kv, int64_t num_blocks, CUtensorMap *lat, CUtensorMap
     e.kv = kv;
     e.num_blocks = num_blocks;
     e.device = dev;
-    cuuint64_t dims[2] = {(cuuint64_t)MLA_D_QK, (cuuint64_t)num_blocks * MLA_BLOCK_TOKENS};
-    cuuint64_t strides[1] = {(cuuint64_t)MLA_D_QK * 2};
-    cuuint32_t box_lat[2] = {64, 64}, box_rope[2] = {32, 64}, estr[2] = {1, 1};
-    if (enc(&e.lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv), dims, strides, box_lat, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    e.fp8 = fp8;
+    const cuuint64_t rows = (cuuint64_t)num_blocks * MLA_BLOCK_TOKENS;
+    const cuuint64_t rec = fp8 ? (cuuint64_t)MLA_FP8_RECORD_BYTES : (cuuint64_t)MLA_D_QK * 2;
+    cuuint64_t dims[2] = {rec / 2, rows};                    // bf16 view
+    cuuint64_t dims8[2] = {rec, rows};                       // uint8 view (fp8 latent)
+    cuuint64_t strides[1] = {rec};
+    cuuint32_t box_lat[2] = {64, 64}, box_lat8[2] = {128, 64}, box_rope[2] = {32, 64}, estr[2] = {1, 1};
+    if (enc(&e.lat, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv),
+            fp8 ? dims8 : dims, strides, fp8 ? box_lat8 : box_lat, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return MLA_ERR_CUDA;
     if (enc(&e.rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv), dims, strides, box_rope, estr,
@@ -176,6 +185,9 @@ DecodeParams make_params(const void *q, const void *kv, int64_t num_blocks, cons
     p.causal = causal;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.v_scale = 1.f;
+    p.q_lat_mul = 1.f;
+    p.q_rope_mul = 1.f;
     return p;
 }
 
@@ -195,6 +207,7 @@ const char *mla_status_string(int status) {
         case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA call failed";
         case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a device pipeline wait hit its bound";
         case MLA_ERR_BOUNDS: return "MLA_ERR_BOUNDS: block-table entry out of range";
+        case MLA_ERR_RANGE: return "MLA_ERR_RANGE: a query value is outside the range of its fp16 form (fp8 cache)";
         default: return "MLA: unknown status";
     }
 }
@@ -256,9 +269,43 @@ int mla_decode_split(const void *q, const void *kv_cache, int64_t num_blocks,
                                  num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
                                  workspace);
     CUtensorMap map_lat, map_rope;
-    rc = cache_maps(kv_cache, num_blocks, &map_lat, &map_rope);
+    rc = cache_maps(kv_cache, num_blocks, 0, &map_lat, &map_rope);
     if (rc != MLA_OK) return rc;
-    cudaError_t e = launch_decode_sm100(p, map_lat, map_rope, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_decode_sm100(p, map_lat, map_rope, false, static_cast<cudaStream_t>(stream));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_blocks, float kv_scale,
+                         const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                         const int32_t *tile_meta, const int32_t *num_splits, int num_parts, int batch,
+                         int s_q, int h_q, float scale, int causal, void *out, float *lse, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    int rc = validate_decode(q, kv_cache_fp8, num_blocks, block_table, bt_stride, seqlens, tile_meta,
+                             num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
+                             workspace, workspace_bytes);
+    if (rc != MLA_OK) return rc;
+    // kv_scale = mu 2^-k with mu in [1, 2): frexp gives kv_scale = f 2^e, f in [0.5, 1)
+    if (!std::isfinite(kv_scale) || !(kv_scale > 0.f)) return MLA_ERR_INVALID_ARG;
+    int e2 = 0;
+    const float f = std::frexp(kv_scale, &e2);
+    const int k = 1 - e2;
+    if (k < -64 || k > 64) return MLA_ERR_INVALID_ARG;
+    const float sl2 = scale * 1.4426950408889634f * std::ldexp(1.f, -k);
+    if (!std::isfinite(sl2)) return MLA_ERR_INVALID_ARG;
+    rc = check_device();
+    if (rc != MLA_OK) return rc;
+    DecodeParams p = make_params(q, kv_cache_fp8, num_blocks, block_table, bt_stride, seqlens, tile_meta,
+                                 num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
+                                 workspace);
+    p.scale_log2 = sl2;
+    p.v_scale = kv_scale;
+    p.q_lat_mul = 2.f * f;
+    p.q_rope_mul = std::ldexp(1.f, k);
+    CUtensorMap map_lat, map_rope;
+    rc = cache_maps(kv_cache_fp8, num_blocks, 1, &map_lat, &map_rope);
+    if (rc != MLA_OK) return rc;
+    cudaError_t e = launch_decode_sm100(p, map_lat, map_rope, true, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -291,6 +338,19 @@ int mla_decode(const void *q, const void *kv_cache, int64_t num_blocks,
     int rc = mla_decode_split(q, kv_cache, num_blocks, block_table, bt_stride, seqlens, tile_meta,
                               num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
                               workspace, workspace_bytes, stream);
+    if (rc != MLA_OK) return rc;
+    return mla_decode_combine(num_splits, num_parts, batch, s_q, h_q, out, lse, workspace,
+                              workspace_bytes, stream);
+}
+
+int mla_decode_fp8(const void *q, const void *kv_cache_fp8, int64_t num_blocks, float kv_scale,
+                   const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                   const int32_t *tile_meta, const int32_t *num_splits, int num_parts, int batch, int s_q,
+                   int h_q, float scale, int causal, void *out, float *lse, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+    int rc = mla_decode_split_fp8(q, kv_cache_fp8, num_blocks, kv_scale, block_table, bt_stride, seqlens,
+                                  tile_meta, num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
+                                  workspace, workspace_bytes, stream);
     if (rc != MLA_OK) return rc;
     return mla_decode_combine(num_splits, num_parts, batch, s_q, h_q, out, lse, workspace,
                               workspace_bytes, stream);
@@ -343,6 +403,7 @@ int mla_check_status(void *stream) {
     if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero) != cudaSuccess) return MLA_ERR_CUDA;
     if (word & kErrBounds) return MLA_ERR_BOUNDS;
     if (word & kErrTimeout) return MLA_ERR_TIMEOUT;
+    if (word & kErrRange) return MLA_ERR_RANGE;
     return MLA_OK;
 }
 

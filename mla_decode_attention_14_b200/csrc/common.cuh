@@ -15,6 +15,7 @@ constexpr int kMetaInts = 8;     // int32 per part in tile_meta
 // Per-device error word (bit flags), read and cleared by mla_check_status().
 constexpr unsigned kErrBounds = 1u;   // a needed block-table entry was outside [0, num_blocks)
 constexpr unsigned kErrTimeout = 2u;  // a pipeline wait hit its iteration bound
+constexpr unsigned kErrRange = 4u;    // fp8 cache: a query value outside the range of its fp16 form
 // Defined here: the library is one translation unit (csrc/mla_lib.cu).
 __device__ unsigned int g_error_word = 0;
 
@@ -37,7 +38,11 @@ struct DecodeParams {
     int batch, s_q, h_q, rows, num_parts;
     int causal;
     float scale;                   // softmax scale
-    float scale_log2;              // scale * log2(e)
+    float scale_log2;              // scale * log2(e) (fp8 cache: also times 2^-k, see q_rope_mul)
+    // fp8 cache only: a latent byte x stands for v_scale * e4m3(x), v_scale = q_lat_mul * 2^-k with
+    // q_lat_mul in [1, 2); the latent query dims are multiplied by q_lat_mul, the rotary ones by
+    // q_rope_mul = 2^k, and the output by v_scale.
+    float v_scale, q_lat_mul, q_rope_mul;
 };
 
 // Visible keys of query token t in a sequence of n tokens (causal: the s_q query

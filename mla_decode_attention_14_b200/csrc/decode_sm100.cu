@@ -50,6 +50,7 @@
 //    kernel; whole sequences are written straight to bf16 out / fp32 lse.
 // Every wait is bounded; a timeout sets the device error word and the CTA exits cleanly.
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -70,6 +71,20 @@ constexpr uint32_t kRegsControl = 96, kRegsSoftmax = 200;
 constexpr int kBoxBytes = kBlk * 128;                      // 64 tokens x 64 bf16 (128-byte swizzle)
 constexpr int kRopeBoxBytes = kBlk * 64;                   // 64 tokens x 32 bf16 (64-byte swizzle)
 constexpr int kStageBytes = 4 * kBoxBytes + kRopeBoxBytes;  // 36,864: half of one cache block
+constexpr int kRingBytes = kStages * kStageBytes;          // shared memory of the KV ring
+// fp8 cache (640-byte token records: 512 E4M3 latent bytes, then 64 bf16 rotary dims): a 4-stage
+// ring of raw half-records (two 64-token x 128-byte latent boxes, 128-byte swizzle, and the rotary
+// box) and, behind it in the same shared memory, 3 buffers of the latent half converted to fp16 in
+// the bf16 stage's layout (four 64 x 64 boxes), which both GEMMs read.
+constexpr int kStages8 = 4, kConvBufs = 3;
+constexpr int kRawBoxBytes = kBlk * 128;                            // 64 tokens x 128 E4M3
+constexpr int kRawStageBytes = 2 * kRawBoxBytes + kRopeBoxBytes;    // 20,480
+constexpr int kConvBytes = 4 * kBoxBytes;                           // 32,768
+constexpr int kConvBase = kStages8 * kRawStageBytes;                // 81,920
+static_assert(kConvBase + kConvBufs * kConvBytes <= kRingBytes, "fp8 ring must fit the bf16 ring");
+template <bool F8> constexpr int ring_stages() { return F8 ? kStages8 : kStages; }
+template <bool F8> constexpr int stage_bytes() { return F8 ? kRawStageBytes : kStageBytes; }
+template <bool F8> constexpr int rope_offset() { return F8 ? 2 * kRawBoxBytes : 4 * kBoxBytes; }
 constexpr float kRescaleThreshold = 8.0f;                  // log2 units: rescale O when max grows > 2^8
 // The pair exchanges R = 2^((s - m) / 2 + 15), the square root of a factor, in fp16: R <= 2^15
 // (< 65504), normal (full 11-bit precision) while s - m >= -58 and subnormal down to -78, so the
@@ -81,24 +96,32 @@ constexpr float kXScaleLog2 = 15.0f;
 constexpr uint32_t kTmemO = 0;     // 256 fp32: O for this CTA's 256 value dims
 constexpr uint32_t kTmemQ = 256;   // 128 x (2 bf16): this CTA's 256 latent query dims
 constexpr uint32_t kTmemS = 384;   // 64 fp32: partial scores of a block
-constexpr uint32_t kTmemPhi = 448; // 32 x (2 bf16): P with its low 16 bits cleared (the A operand of Gemm2)
-constexpr uint32_t kTmemPlo = 480; // 32 x (2 bf16): the remainder, likewise
+constexpr uint32_t kTmemPhi = 448; // 32 x (2 bf16): P with its low 16 bits cleared (the A operand of Gemm2);
+                                   // fp8 cache: P as fp16 (the only term)
+constexpr uint32_t kTmemPlo = 480; // 32 x (2 bf16): the remainder, likewise (bf16 cache only)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kXchgEBytes = 2 * kBlk * 128 * 2;    // two slots of 128 rows x 64 fp16 factors
 constexpr int kXchgOffBytes = 2 * kTq * 128 * 4;   // two slots of 128 rows x 2 fp32 offsets
 
 struct __align__(1024) Smem {
-    uint8_t stage[kStages][kStageBytes];  // KV ring
+    uint8_t ring[kRingBytes];  // KV ring (bf16: kStages stages; fp8: raw stages, then fp16 buffers)
     uint4 xchg[(kXchgEBytes + kXchgOffBytes) / 16];  // peer factors R (fp16) [slot][token half][16 B][row]
                                                      // + row offsets (fp32) [slot][token half][row]
     float xmax[2][kTq][128];  // per-row exchange between the two token halves (block max bound; sums)
     uint8_t q_rope[128 * 64];             // rotary query dims [128 rows x 32], K-major, 64-byte swizzle
     uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t conv_full[kConvBufs], conv_empty[kConvBufs];  // fp8 cache: converted latent buffers
     uint64_t s_full, s_free, p_full, p_free, o_full, o_free, q_full, mma_done;
     uint64_t xfull[2];  // receive slots filled by the peer
     uint32_t tmem_base;
     int abort;
 };
+
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory (with 1 KB for alignment) must fit 227 KB");
+
+template <bool F8>
+__device__ __forceinline__ uint8_t *stage_ptr(Smem &sm, int s) { return sm.ring + s * stage_bytes<F8>(); }
+__device__ __forceinline__ uint8_t *conv_ptr(Smem &sm, int c) { return sm.ring + kConvBase + c * kConvBytes; }
 
 struct Piece {
     int seq, lo, hi, n, nsplit, slot;
@@ -166,15 +189,17 @@ struct BlockWalker {
 };
 
 // ---------------------------------------------------------------- TMA producer (1 thread)
+template <bool F8>
 __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map_lat, const CUtensorMap *map_rope,
                          const int32_t *meta, uint32_t half) {
+    constexpr int NS = ring_stages<F8>();
     const uint64_t policy = l2_evict_first_policy();
     BlockWalker w;
     w.init(meta, p);
     int gidx = 0;
     bool bad_block = false;
     for (; w.live; w.advance(p), ++gidx) {
-        const int s = gidx % kStages, fill = gidx / kStages;
+        const int s = gidx % NS, fill = gidx / NS;
         if (fill > 0 && !mbar_wait(&sm.kv_empty[s], (fill - 1) & 1, &sm.abort)) break;
         const int phys = w.blk < p.bt_stride ? __ldg(&p.block_table[(size_t)w.pc.seq * p.bt_stride + w.blk]) : -1;
         if (phys < 0 || (int64_t)phys >= p.num_blocks) {
@@ -182,19 +207,26 @@ __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map
             mbar_arrive(&sm.kv_full[s]);  // consumers run on stale data; the error word reports it
             continue;
         }
-        mbar_arrive_expect_tx(&sm.kv_full[s], kStageBytes);
+        mbar_arrive_expect_tx(&sm.kv_full[s], stage_bytes<F8>());
         const int y = phys * kBlk;
-        uint8_t *dst = sm.stage[s];
+        uint8_t *dst = stage_ptr<F8>(sm, s);
+        if constexpr (F8) {  // coordinates: bytes of the record (latent), bf16 elements (rotary)
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
-            tma_load_2d(dst + b * kBoxBytes, map_lat, 256 * (int)half + 64 * b, y, &sm.kv_full[s], policy);
-        tma_load_2d(dst + 4 * kBoxBytes, map_rope, 512 + 32 * (int)half, y, &sm.kv_full[s], policy);
+            for (int b = 0; b < 2; ++b)
+                tma_load_2d(dst + b * kRawBoxBytes, map_lat, 256 * (int)half + 128 * b, y, &sm.kv_full[s], policy);
+            tma_load_2d(dst + rope_offset<F8>(), map_rope, 256 + 32 * (int)half, y, &sm.kv_full[s], policy);
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                tma_load_2d(dst + b * kBoxBytes, map_lat, 256 * (int)half + 64 * b, y, &sm.kv_full[s], policy);
+            tma_load_2d(dst + rope_offset<F8>(), map_rope, 512 + 32 * (int)half, y, &sm.kv_full[s], policy);
+        }
     }
     if (bad_block) raise_error(kErrBounds);
     // every load still in flight must land before the CTA may exit
-    for (int k = max(0, gidx - kStages); k < gidx; ++k) {
+    for (int k = max(0, gidx - NS); k < gidx; ++k) {
         const long long t0 = clock64();
-        while (!mbar_sleep_test(&sm.kv_full[k % kStages], (k / kStages) & 1) && clock64() - t0 < kSpinCycles) {
+        while (!mbar_sleep_test(&sm.kv_full[k % NS], (k / NS) & 1) && clock64() - t0 < kSpinCycles) {
         }
     }
 }
@@ -221,44 +253,105 @@ __device__ void zero_tail_rows(uint8_t *st, int valid, int lane) {
     __syncwarp();
 }
 
+// fp8 cache, warp 2: the latent half of every block from E4M3 to fp16 -- exact, every E4M3 value is
+// an fp16 number -- into a buffer in the layout the MMA descriptors read (the bf16 stage's four
+// 128-byte-swizzled boxes of 64 tokens x 64 dims). Rows past a sequence's end are written as zeros,
+// so undefined tail contents never reach Gemm2. Lane mapping: each group of 8 lanes takes 16-byte
+// chunks 0-3 of one row of a row pair and chunks 4-7 of the other row, so the group's reads (one
+// chunk each) and writes (two chunks each) both fall on 8 distinct 16-byte bank groups.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+__device__ void convert_warp(Smem &sm, const DecodeParams &p, const int32_t *meta) {
+    const int lane = threadIdx.x & 31;
+    const int u = lane & 7, hp = (lane >> 3) & 1, pq = lane >> 4;  // chunk, half of the pair, pair of the step
+    const int k0 = 2 * (u & 3);                                     // first fp16 chunk of the box row
+    volatile int *abort = &sm.abort;
+    BlockWalker w;
+    w.init(meta, p);
+    for (int g = 0; w.live; w.advance(p), ++g) {
+        const int s = g % kStages8, c = g % kConvBufs;
+        if (!warp_wait(&sm.kv_full[s], (g / kStages8) & 1, abort, lane)) break;
+        if (g >= kConvBufs && !warp_wait(&sm.conv_empty[c], (g / kConvBufs - 1) & 1, abort, lane)) break;
+        const int valid = w.tail() ? w.pc.n - w.blk * kBlk : kBlk;
+        const uint8_t *raw = stage_ptr<true>(sm, s);
+        uint8_t *dst = conv_ptr(sm, c);
+#pragma unroll 4
+        for (int it = 0; it < 32; ++it) {
+            const int pi = 2 * it + pq;  // row pair over both raw boxes: 2 x 32 pairs
+            const int bx = pi >> 5, row = 2 * (pi & 31) + ((u >> 2) ^ hp), sw = row & 7;
+            uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+            if (row < valid) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(raw + bx * kRawBoxBytes + row * 128 + ((u ^ sw) << 4));
+                lo = make_uint4(e4m3x2_to_f16x2(x.x & 0xffffu), e4m3x2_to_f16x2(x.x >> 16),
+                                e4m3x2_to_f16x2(x.y & 0xffffu), e4m3x2_to_f16x2(x.y >> 16));
+                hi = make_uint4(e4m3x2_to_f16x2(x.z & 0xffffu), e4m3x2_to_f16x2(x.z >> 16),
+                                e4m3x2_to_f16x2(x.w & 0xffffu), e4m3x2_to_f16x2(x.w >> 16));
+            }
+            uint8_t *o = dst + (2 * bx + (u >> 2)) * kBoxBytes + row * 128;
+            *reinterpret_cast<uint4 *>(o + ((k0 ^ sw) << 4)) = lo;
+            *reinterpret_cast<uint4 *>(o + (((k0 + 1) ^ sw) << 4)) = hi;
+        }
+        fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&sm.conv_full[c]);
+            mbar_arrive(&sm.kv_empty[s]);  // the raw latent is consumed (Gemm1 still reads the rotary box)
+        }
+    }
+}
+
 // Issuing one tcgen05 MMA occupies the issuing thread for about 70 cycles whatever its size, so
 // Gemm1 and Gemm2 are issued by two warps: the tensor core takes MMAs from both at once.
 
 // Gemm1 of every block into S (partial scores over this CTA's 288 dims): 18 MMAs into one
 // accumulator; the next block's Gemm1 may start as soon as the softmax warps have read S.
+// fp8 cache: the 16 latent MMAs are fp16 x fp16 (Q converted on load, K from the converted
+// buffer), the 2 rotary MMAs stay bf16 x bf16 from the raw stage; both accumulate in fp32.
+template <bool F8>
 __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
     constexpr uint32_t id1 = idesc_bf16_f32(128, 64, 0);  // S = Q K^T: K-major B
+    constexpr uint32_t id1_lat = F8 ? idesc_f16_f32(128, 64, 0) : id1;
+    constexpr int NS = ring_stages<F8>();
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
     BlockWalker w;
     w.init(meta, p);
     for (int g = 0; w.live; w.advance(p), ++g) {
         if (w.first() && !warp_wait(&sm.q_full, w.piece_k & 1, abort, lane)) break;
-        const int s = g % kStages;
-        if (!warp_wait(&sm.kv_full[s], (g / kStages) & 1, abort, lane)) break;
+        const int s = g % NS, cb = g % kConvBufs;
+        if (!warp_wait(&sm.kv_full[s], (g / NS) & 1, abort, lane)) break;
+        if (F8 && !warp_wait(&sm.conv_full[cb], (g / kConvBufs) & 1, abort, lane)) break;
         if (g > 0 && !warp_wait(&sm.s_free, (g - 1) & 1, abort, lane)) break;
         if (lane == 0) {
             tc_fence_after();
             // descriptors: one base each, then constant offsets (address field is in 16-byte units)
-            const uint64_t kd = smem_desc(smem_addr(sm.stage[s]), 16, 1024, 2);
-            const uint64_t rd = smem_desc(smem_addr(sm.stage[s]) + 4 * kBoxBytes, 16, 512, 4);
+            const uint8_t *lat = F8 ? conv_ptr(sm, cb) : stage_ptr<F8>(sm, s);
+            const uint64_t kd = smem_desc(smem_addr(lat), 16, 1024, 2);
+            const uint64_t rd = smem_desc(smem_addr(stage_ptr<F8>(sm, s)) + rope_offset<F8>(), 16, 512, 4);
             const uint64_t qd = smem_desc(smem_addr(sm.q_rope), 16, 512, 4);
 #pragma unroll
             for (int k = 0; k < 16; ++k)  // latent k-steps, A (Q) from TMEM
                 mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * k, kd + (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4),
-                       id1, k > 0 ? 1u : 0u);
+                       id1_lat, k > 0 ? 1u : 0u);
 #pragma unroll
             for (int c = 0; c < 2; ++c)  // rotary k-steps, A from shared memory
                 mma_ss(tmem + kTmemS, qd + 2 * c, rd + 2 * c, id1, 1u);
             mma_commit(&sm.s_full);
+            if (F8) mma_commit(&sm.kv_empty[s]);  // the raw stage's rotary box is consumed
         }
         __syncwarp();
     }
 }
 
 // Gemm2 of every block, O (+)= (P_hi + P_lo) V, once the softmax warps have written P.
+// fp8 cache: O (+)= P V with P and V in fp16, 4 MMAs.
+template <bool F8>
 __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
-    constexpr uint32_t id2 = idesc_bf16_f32(128, 256, 1);  // MN-major B
+    constexpr uint32_t id2 = F8 ? idesc_f16_f32(128, 256, 1) : idesc_bf16_f32(128, 256, 1);  // MN-major B
+    constexpr int NS = ring_stages<F8>(), kTerms = F8 ? 1 : 2;
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
     BlockWalker w;
@@ -266,21 +359,22 @@ __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
     for (int g = 0; w.live; w.advance(p), ++g) {
         if (!warp_wait(&sm.p_full, g & 1, abort, lane)) break;
         if (w.first() && w.piece_k > 0 && !warp_wait(&sm.o_free, (w.piece_k - 1) & 1, abort, lane)) break;
-        const int s = g % kStages;
-        // P of block g exists, so Gemm1 of block g has completed and its tile may be edited
-        if (w.tail()) zero_tail_rows(sm.stage[s], w.pc.n - w.blk * kBlk, lane);
+        const int s = g % NS, cb = g % kConvBufs;
+        // P of block g exists, so Gemm1 of block g has completed and its tile may be edited (the fp8
+        // path's converter has already zeroed the tail rows)
+        if (!F8 && w.tail()) zero_tail_rows(stage_ptr<F8>(sm, s), w.pc.n - w.blk * kBlk, lane);
         if (lane == 0) {
             tc_fence_after();
-            const uint64_t vd = smem_desc(smem_addr(sm.stage[s]), 4 * 2048, 1024, 2);
+            const uint64_t vd = smem_desc(smem_addr(F8 ? conv_ptr(sm, cb) : stage_ptr<F8>(sm, s)), 4 * 2048, 1024, 2);
             const bool first = w.first();
 #pragma unroll
-            for (int hl = 0; hl < 2; ++hl)  // P_hi, then P_lo, A from TMEM
+            for (int hl = 0; hl < kTerms; ++hl)  // P_hi, then P_lo, A from TMEM
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_ts(tmem + kTmemO, tmem + (hl ? kTmemPlo : kTmemPhi) + 8 * kk, vd + 128 * kk, id2,
                            (!first || hl > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&sm.p_free);
-            mma_commit(&sm.kv_empty[s]);
+            mma_commit(F8 ? &sm.conv_empty[cb] : &sm.kv_empty[s]);
             if (w.last()) mma_commit(&sm.o_full);
         }
         __syncwarp();
@@ -309,11 +403,31 @@ struct SoftCtx {
     bool row_ok, warp_ok;
 };
 
+// fp8 cache: a bf16 pair times `mul` as an fp16 pair (round to nearest); flags values past the fp16
+// range (or not finite).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, float mul, bool &bad) {
+    const float a = __uint_as_float(v << 16) * mul, b = __uint_as_float(v & 0xffff0000u) * mul;
+    bad |= !(fabsf(a) <= 65504.f) || !(fabsf(b) <= 65504.f);
+    __half2 two = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&two);
+}
+// A bf16 pair times a power of two (exact unless it leaves the range; flags overflow).
+__device__ __forceinline__ uint32_t bf16x2_pow2(uint32_t v, float pow2, bool &bad) {
+    const float a = __uint_as_float(v << 16) * pow2, b = __uint_as_float(v & 0xffff0000u) * pow2;
+    bad |= !(fabsf(a) <= 3.0e38f) || !(fabsf(b) <= 3.0e38f);
+    return (__float_as_uint(a) >> 16) | (__float_as_uint(b) & 0xffff0000u);
+}
+
 // Q of piece `pc`: latent half -> TMEM (this warp's lanes, its 64 of the 128 columns),
 // rotary half -> shared memory (its 2 of the 4 16-byte chunks of the row).
+// fp8 cache, with the latent scale written as mu 2^-k (mu in [1, 2)): the latent dims go to TMEM
+// as fp16(q mu) and the rotary dims as q 2^k (exact), so that the accumulated score is 2^k times
+// scale^-1 s; the kernel's score scale carries the 2^-k.
+template <bool F8>
 __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &pc) {
     if (c.warp_ok) {
         const DecodeParams &p = *c.p;
+        bool bad = false;
         const uint4 *qrow =
             reinterpret_cast<const uint4 *>(p.q + ((size_t)pc.seq * p.rows + (c.row_ok ? c.r : 0)) * kDqk);
 #pragma unroll 1
@@ -327,13 +441,21 @@ __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &
                 w[4 * v + 2] = x.z;
                 w[4 * v + 3] = x.w;
             }
+            if constexpr (F8) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) w[k] = bf16x2_to_f16x2(w[k], p.q_lat_mul, bad);
+            }
             tmem_st16(c.tmem + kTmemQ + c.lane_off + 16 * c16, w);
         }
 #pragma unroll
         for (int v = 2 * c.th; v < 2 * c.th + 2; ++v) {  // rotary dims: 16-byte chunks, 64-byte swizzle
-            const uint4 x = c.row_ok ? __ldg(qrow + (512 + 32 * (int)c.half) / 8 + v) : make_uint4(0, 0, 0, 0);
+            uint4 x = c.row_ok ? __ldg(qrow + (512 + 32 * (int)c.half) / 8 + v) : make_uint4(0, 0, 0, 0);
+            if constexpr (F8)
+                x = make_uint4(bf16x2_pow2(x.x, p.q_rope_mul, bad), bf16x2_pow2(x.y, p.q_rope_mul, bad),
+                               bf16x2_pow2(x.z, p.q_rope_mul, bad), bf16x2_pow2(x.w, p.q_rope_mul, bad));
             *reinterpret_cast<uint4 *>(sm.q_rope + c.i * 64 + ((v ^ ((c.i >> 1) & 3)) * 16)) = x;
         }
+        if (F8 && bad) raise_error(kErrRange);
         tmem_wait_st();
         fence_proxy_async_smem();
     }
@@ -406,6 +528,7 @@ __device__ __forceinline__ float exps_in_place(float (&s)[kTokPer], float sl2) {
     return m;
 }
 
+template <bool F8>
 __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem, uint32_t half,
                              int group) {
     SoftCtx c;
@@ -438,7 +561,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     BlockWalker w;
     w.init(meta, p);
     if (!w.live) return;
-    load_q(sm, c, w.pc);
+    load_q<F8>(sm, c, w.pc);
     int vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
     float e_own[kTokPer], m_own;
     if (!load_raw(sm, c, 0, w.blk * kBlk, vis, e_own)) return;
@@ -447,7 +570,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     if (w.last()) {  // the next piece's Q may replace this one once its last Gemm1 is done
         Cursor tmp = w.cur;
         Piece nx;
-        if (tmp.next(p, nx)) load_q(sm, c, nx);
+        if (tmp.next(p, nx)) load_q<F8>(sm, c, nx);
     }
     float m_ref = -INFINITY, l = 0.f;
     for (int g = 0; w.live; ++g) {
@@ -464,7 +587,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
             if (w.last()) {
                 Cursor tmp = w.cur;
                 Piece nx;
-                if (tmp.next(p, nx)) load_q(sm, c, nx);
+                if (tmp.next(p, nx)) load_q<F8>(sm, c, nx);
             }
         } else {
 #pragma unroll
@@ -475,11 +598,45 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         if (threadIdx.x == 32 * kFirstSoftWarp) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
         if (!mbar_wait_cluster(&sm.xfull[slot], (g >> 1) & 1, abort)) return;
         const float m_peer = c.warp_ok ? xo[(slot * kTq + c.th) * 128 + c.i] : -INFINITY;
-        // an upper bound of the block's row max (both token halves), shared by the two warps of a row
         const float mbu_half = m_own + m_peer;
-        sm.xmax[g & 1][c.th][c.i] = mbu_half;
-        named_bar_sync(bar_id, 64);
-        const float mbu = fmaxf(mbu_half, sm.xmax[g & 1][c.th ^ 1][c.i]);
+        uint32_t ep[kTokPer / 2];  // the peer's factors, fp16 pairs
+        float mbu;                 // the block's row max (both token halves), shared by the two warps of a row
+        if constexpr (F8) {
+            // exact: t_j = R_own R_peer = 2^((s_j - m_own - m_peer) / 2 + 30) in place of R_own, and
+            // the max of t gives the max of s. fp16 P needs it: an upper bound that overstates the
+            // max by o octaves would leave P below 2^-o, where fp16 loses precision.
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const uint4 v = xe[((slot * kTq + c.th) * 4 + c4) * 128 + c.i];
+                ep[4 * c4] = v.x;
+                ep[4 * c4 + 1] = v.y;
+                ep[4 * c4 + 2] = v.z;
+                ep[4 * c4 + 3] = v.w;
+            }
+            float t[16];
+#pragma unroll
+            for (int j = 0; j < kTokPer; j += 2) {
+                const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
+                e_own[j] *= e2.x;
+                e_own[j + 1] *= e2.y;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) t[j] = fmaxf(e_own[j], e_own[j + 16]);
+#pragma unroll
+            for (int k = 8; k >= 1; k >>= 1)
+#pragma unroll
+                for (int j = 0; j < k; ++j) t[j] = fmaxf(t[j], t[j + k]);
+            const float mx_half =
+                (t[0] > 0.f && mbu_half != -INFINITY) ? 2.f * (__log2f(t[0]) - 2.f * kXScaleLog2) + mbu_half : -INFINITY;
+            sm.xmax[g & 1][c.th][c.i] = mx_half;
+            named_bar_sync(bar_id, 64);
+            mbu = fmaxf(mx_half, sm.xmax[g & 1][c.th ^ 1][c.i]);
+        } else {
+            // an upper bound of the block's row max
+            sm.xmax[g & 1][c.th][c.i] = mbu_half;
+            named_bar_sync(bar_id, 64);
+            mbu = fmaxf(mbu_half, sm.xmax[g & 1][c.th ^ 1][c.i]);
+        }
         bool need = false;
         float alpha = 1.f;
         if (a_first) {
@@ -495,14 +652,15 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 need = true;
             }
         }
-        uint32_t ep[kTokPer / 2];  // the peer's factors, fp16 pairs
+        if constexpr (!F8) {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const uint4 v = xe[((slot * kTq + c.th) * 4 + c4) * 128 + c.i];
-            ep[4 * c4] = v.x;
-            ep[4 * c4 + 1] = v.y;
-            ep[4 * c4 + 2] = v.z;
-            ep[4 * c4 + 3] = v.w;
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const uint4 v = xe[((slot * kTq + c.th) * 4 + c4) * 128 + c.i];
+                ep[4 * c4] = v.x;
+                ep[4 * c4 + 1] = v.y;
+                ep[4 * c4 + 2] = v.z;
+                ep[4 * c4 + 3] = v.w;
+            }
         }
         // One straight-line region: P of block g (FMA and ALU work), the exponentials of block g+1
         // (MUFU work) and their stores into the peer (distributed shared memory, ~20 bytes per
@@ -544,14 +702,21 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 __half2 two = __floats2half2_rn(snx[j], snx[j + 1]);
                 wv[q] = *reinterpret_cast<uint32_t *>(&two);
                 // P of block g
-                const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
-                const float t0 = e_own[j] * e2.x, t1 = e_own[j + 1] * e2.y;
-                const float p0 = t0 * t0 * f, p1 = t1 * t1 * f;
-                su[q] += p0 + p1;
-                const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-                const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
-                pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
-                pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                if constexpr (F8) {  // e_own holds t = R_own R_peer; P in fp16 (round to nearest)
+                    const float p0 = e_own[j] * e_own[j] * f, p1 = e_own[j + 1] * e_own[j + 1] * f;
+                    su[q] += p0 + p1;
+                    __half2 ph = __floats2half2_rn(p0, p1);
+                    pk[j >> 1] = *reinterpret_cast<uint32_t *>(&ph);
+                } else {
+                    const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
+                    const float t0 = e_own[j] * e2.x, t1 = e_own[j + 1] * e2.y;
+                    const float p0 = t0 * t0 * f, p1 = t1 * t1 * f;
+                    su[q] += p0 + p1;
+                    const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                    const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                    pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
+                    pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                }
             }
             if (send) st_async_v4_b32(xbase + c4 * 128 * 16, wv[0], wv[1], wv[2], wv[3], xbar);
         }
@@ -577,7 +742,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         }
         // this thread's 32 tokens of row i in both P regions of TMEM (bf16 pairs, lane = row)
         tmem_st16(tmem + kTmemPhi + c.lane_off + 16 * c.th, pk);
-        tmem_st16(tmem + kTmemPlo + c.lane_off + 16 * c.th, pl);
+        if constexpr (!F8) tmem_st16(tmem + kTmemPlo + c.lane_off + 16 * c.th, pl);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -593,7 +758,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
             tc_fence_after();
             if (c.warp_ok) {
                 const bool empty = !(l_row > 0.f);
-                const float inv = empty ? 0.f : 1.f / l_row;
+                const float inv = empty ? 0.f : (F8 ? p.v_scale / l_row : 1.f / l_row);
                 const bool whole = a_nsplit == 1;
 #pragma unroll 1
                 for (int q = 0; q < 8; ++q) {
@@ -647,6 +812,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     }
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_rope,
                     const DecodeParams p, const int groups) {
@@ -662,7 +828,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.kv_empty[s], F8 ? 2 : 1);  // fp8: the converter and Gemm1's commit
+        }
+        for (int b = 0; b < kConvBufs; ++b) {
+            mbar_init(&sm.conv_full[b], 1);
+            mbar_init(&sm.conv_empty[b], 1);
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.s_free, kSoftWarps);
@@ -690,19 +860,21 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     if (warp < kFirstSoftWarp) {
         setmaxnreg_dec<kRegsControl>();
         if (warp == 0) {
-            if (lane == 0) producer(sm, p, &map_lat, &map_rope, meta, half);
+            if (lane == 0) producer<F8>(sm, p, &map_lat, &map_rope, meta, half);
         } else {
             if (warp == 3) {
-                gemm2_warp(sm, p, meta, tmem);
+                gemm2_warp<F8>(sm, p, meta, tmem);
                 drain_mmas(sm);
             } else if (warp == 1) {
-                gemm1_warp(sm, p, meta, tmem);
+                gemm1_warp<F8>(sm, p, meta, tmem);
                 drain_mmas(sm);
+            } else if (F8) {
+                convert_warp(sm, p, meta);
             }
         }
     } else {
         setmaxnreg_inc<kRegsSoftmax>();
-        softmax_role(sm, p, meta, tmem, half, group);
+        softmax_role<F8>(sm, p, meta, tmem, half, group);
     }
     __syncwarp();
     tc_fence_before();
@@ -720,11 +892,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
 size_t decode_sm100_smem_bytes() { return sizeof(dec::Smem) + 1024; }
 
 cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
-                                cudaStream_t stream) {
+                                bool fp8, cudaStream_t stream) {
     const int groups = (p.rows + 127) / 128;
     const size_t smem = decode_sm100_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(dec::decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    auto kernel = fp8 ? dec::decode_sm100_kernel<true> : dec::decode_sm100_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * p.num_parts * groups, 1, 1);
@@ -738,7 +910,7 @@ cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_la
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, dec::decode_sm100_kernel, map_lat, map_rope, p, groups);
+    return cudaLaunchKernelEx(&cfg, kernel, map_lat, map_rope, p, groups);
 }
 
 }  // namespace mla

@@ -137,6 +137,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn) {
            ((uint32_t)(M >> 4) << 24);
 }
 
+// The same for fp16 A and B (format fields 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int b_mn) {
+    return (1u << 4) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]
 MLA_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
