@@ -2,6 +2,7 @@
 """Benchmark of MLA decode attention on B200: effective TB/s (KV + Q bytes) and TFLOPS.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3] [--impl ours|reference]
+                    [--kv bf16|fp8]
 
 One step = the whole decode path for one batch: split-KV metadata, the split kernel and
 the combine kernel, on inputs already resident in HBM. Where the inputs are larger than
@@ -12,6 +13,9 @@ prints one JSON line.
 Multi-GPU: one process per GPU (torchrun); every rank decodes its own batch of the same
 shape (independent problems, no collective on the data path: weak scaling); the time is
 the max over ranks and the value counts the bytes of all ranks.
+
+``--kv fp8`` runs the same workload over the fp8 (E4M3) latent cache (640 bytes per token);
+the bytes of the metric are then the fp8 cache's.
 
 ``--impl reference`` times the CPU oracle (the plain C fp64 implementation under
 ``oracle/``) on a bounded sample of the same workload; it is the deliberately slow
@@ -39,15 +43,33 @@ from mla_decode_attention_14_b200 import workloads as W  # noqa: E402
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 METRIC = "MLA decode effective TB/s and TFLOPS vs B200 roofline (bf16 paged KV)"
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_split_v3_traffic.txt")
+METRIC_FP8 = "MLA decode effective TB/s and TFLOPS vs B200 roofline (fp8 paged KV)"
+PROFILE_TRAFFIC = {"bf16": os.path.join(ROOT, "profiles", "decode_split_v3_traffic.txt"),
+                   "fp8": os.path.join(ROOT, "profiles", "decode_split_fp8_v3_traffic.txt")}
 L2_BYTES = 126 << 20
 
 
-def describe(wl: W.Workload) -> str:
+def describe(wl: W.Workload, kv: str = "bf16") -> str:
     n = wl.seqlens
+    cache = ("bf16 N(0,1)" if kv == "bf16" else
+             "fp8 cache: E4M3 latent (N(0,1) x 64, latent scale 2^-6) + bf16 N(0,1) rotary, 640 B/token; bf16 N(0,1) q")
     return ("%s: batch %d, h_q %d, s_q %d%s, seqlens %d..%d (mean %.0f), 64-token blocks, d_qk 576, d_v 512, "
-            "bf16 N(0,1), scale 192^-0.5" % (wl.name, wl.batch, wl.h_q, wl.s_q, " causal" if wl.causal else "",
-                                             n.min(), n.max(), n.mean()))
+            "%s, scale 192^-0.5" % (wl.name, wl.batch, wl.h_q, wl.s_q, " causal" if wl.causal else "",
+                                    n.min(), n.max(), n.mean(), cache))
+
+
+def kv_token_bytes(kv: str) -> int:
+    return W.F8_REC if kv == "fp8" else 2 * W.D_QK
+
+
+def oracle_decode(kv, inp, wl, tasks, nthreads):
+    """The oracle over the run's cache format (test infrastructure: the CPU-baseline leg only)."""
+    import oracle
+    if kv == "fp8":
+        return oracle.decode_fp8(inp["q"], inp["kv8"], inp["kv_scale"], inp["block_table"], inp["seqlens"],
+                                 wl.scale, wl.causal, tasks=tasks, nthreads=nthreads)
+    return oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
+                         tasks=tasks, nthreads=nthreads)
 
 
 def measured_peaks():
@@ -79,12 +101,12 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def profiled_traffic(cache: str = "bf16"):
     """DRAM bytes per split-kernel launch from the committed ncu summary, if it was taken
     on the current kernel sources (else None)."""
     try:
         kv = {}
-        with open(PROFILE_TRAFFIC) as f:
+        with open(PROFILE_TRAFFIC[cache]) as f:
             for line in f:
                 if ":" in line and not line.startswith("#"):
                     k, v = line.split(":", 1)
@@ -168,7 +190,6 @@ def job_throughput(bytes_per_rank: int, world: int, ms_per_step: float) -> float
 
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, wl, inp, counts):
-    import oracle
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -177,8 +198,7 @@ def run_reference(args, wl, inp, counts):
     # calibrate: one row of the longest sequence
     b_long = int(np.argmax(wl.seqlens))
     t0 = time.perf_counter()
-    oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
-                  tasks=np.array([[b_long, 0, 0]], np.int32), nthreads=1)
+    oracle_decode(args.kv, inp, wl, np.array([[b_long, 0, 0]], np.int32), 1)
     per_row = max(time.perf_counter() - t0, 1e-4) * float(wl.seqlens.mean()) / float(wl.seqlens.max())
     budget = min(10.0, 150.0 / max(1, args.steps + args.warmup))      # seconds of wall time per step
     nrows = int(max(1, min(wl.h_q * wl.s_q, budget * cores / per_row)))
@@ -187,31 +207,29 @@ def run_reference(args, wl, inp, counts):
     tasks = np.array([[seq, (i // wl.h_q) % wl.s_q, h] for i, h in enumerate(heads)], np.int32)
     n = int(wl.seqlens[seq])
     # algorithmic bytes of this sample: the sequence's KV once, plus its sampled query rows
-    sample_bytes = n * 1152 + nrows * 1152
+    sample_bytes = n * kv_token_bytes(args.kv) + nrows * 1152
     for _ in range(args.warmup):
-        oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
-                      tasks=tasks, nthreads=cores)
+        oracle_decode(args.kv, inp, wl, tasks, cores)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
-                      tasks=tasks, nthreads=cores)
+        oracle_decode(args.kv, inp, wl, tasks, cores)
     dt = (time.perf_counter() - t0) / args.steps
     tbs = sample_bytes / dt / 1e12
     sample = "%d of %d query rows of sequence %d (%d tokens), all its keys, per step" % (nrows, wl.rows, seq, n)
-    line = {"metric": METRIC, "value": tbs, "unit": "TB/s", "n_gpus": args.gpus, "steps": args.steps,
+    line = {"metric": METRIC_FP8 if args.kv == "fp8" else METRIC, "value": tbs, "unit": "TB/s",
+            "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": describe(wl), "sample": sample},
+            "config": {"workload": describe(wl, args.kv), "kv": args.kv, "sample": sample},
             "cpu_baseline": {"value": tbs, "unit": "TB/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": tbs, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # --------------------------------------------------------------------------- our arm
-def cpu_baseline(wl, inp, target_s=12.0):
+def cpu_baseline(wl, inp, target_s=12.0, kv="bf16"):
     """The oracle, as it stands, on a bounded sample of the workload (rank 0, N = 1): whole
     sequences (every query row, every key) in a seeded order until ~target_s of CPU work."""
-    import oracle
     cores = os.cpu_count() or 1
     order = np.random.default_rng(0).permutation(wl.batch)
 
@@ -219,8 +237,7 @@ def cpu_baseline(wl, inp, target_s=12.0):
         return np.array([[s, t, h] for s in seqs for t in range(wl.s_q) for h in range(wl.h_q)], np.int32)
 
     t0 = time.perf_counter()
-    oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
-                  tasks=rows_of([int(order[0])]), nthreads=cores)
+    oracle_decode(kv, inp, wl, rows_of([int(order[0])]), cores)
     per_token = max(time.perf_counter() - t0, 1e-6) / max(1, int(wl.seqlens[order[0]]))
     chosen, est = [], 0.0
     for s in order:
@@ -229,12 +246,11 @@ def cpu_baseline(wl, inp, target_s=12.0):
         if est >= target_s:
             break
     t0 = time.perf_counter()
-    oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, wl.causal,
-                  tasks=rows_of(chosen), nthreads=cores)
+    oracle_decode(kv, inp, wl, rows_of(chosen), cores)
     dt = time.perf_counter() - t0
     n = int(sum(int(wl.seqlens[s]) for s in chosen))
     # the metric's unit: algorithmic bytes (each sampled sequence's KV once + its query rows) per second
-    val = (n * 1152 + len(chosen) * wl.rows * 1152) / dt / 1e12
+    val = (n * kv_token_bytes(kv) + len(chosen) * wl.rows * 1152) / dt / 1e12
     return {"value": val, "unit": "TB/s", "cores": cores, "kind": "oracle",
             "sample": "%d of %d sequences (%d tokens, all %d query rows each), %.1f s on %d threads"
                       % (len(chosen), wl.batch, n, wl.rows, dt, cores),
@@ -248,6 +264,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="v3", choices=W.NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="cache format: bf16 (576 dims) or fp8 (E4M3 latent + bf16 rotary, 640 B/token)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--graph-steps", type=int, default=-1,
                     help="replays of the step captured in a CUDA graph, reported under 'graph' "
@@ -263,7 +281,11 @@ def main():
     if args.max_batch and args.max_batch < wl.batch:
         wl = W.custom(args.max_batch, wl.h_q, wl.s_q, wl.seqlens[:args.max_batch], wl.causal, wl.scale,
                       name="%s[:%d]" % (wl.name, args.max_batch))
-    counts = W.algorithmic_counts(wl)
+    counts = W.algorithmic_counts(wl, kv=args.kv)
+    fp8 = args.kv == "fp8"
+
+    def make_inputs():
+        return W.make_inputs_fp8(wl, seed=0, tail="normal") if fp8 else W.make_inputs(wl, seed=0, tail="normal")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -272,7 +294,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        inp = W.make_inputs(wl, seed=0, tail="normal")
+        inp = make_inputs()
         run_reference(args, wl, inp, counts)
         return
 
@@ -288,10 +310,10 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    inp = W.make_inputs(wl, seed=0, tail="normal")
+    inp = make_inputs()
     dev = torch.device("cuda", local)
     q = torch.from_numpy(inp["q"]).view(torch.bfloat16).to(dev)
-    kv = torch.from_numpy(inp["kv"]).view(torch.bfloat16).to(dev)
+    kv = (torch.from_numpy(inp["kv8"]) if fp8 else torch.from_numpy(inp["kv"]).view(torch.bfloat16)).to(dev)
     bt = torch.from_numpy(inp["block_table"]).to(dev)
     sl = torch.from_numpy(inp["seqlens"]).to(dev)
     num_parts = mla.default_num_parts(wl.h_q, wl.s_q, dev)
@@ -301,14 +323,20 @@ def main():
     lse = torch.empty((wl.batch, wl.h_q, wl.s_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def decode(q, kv, bt, sl, meta, out, lse, ws, phase):
+        if fp8:
+            return mla.decode_fp8(q, kv, bt, sl, wl.scale, inp["kv_scale"], wl.causal, meta, out=out, lse=lse,
+                                  workspace=ws, phase=phase)
+        return mla.decode(q, kv, bt, sl, wl.scale, wl.causal, meta, out=out, lse=lse, workspace=ws, phase=phase)
+
     def step(ev=None):
         meta = mla.get_metadata(sl, wl.h_q, wl.s_q, num_parts=num_parts, fixed_cost=fixed_cost)
         if ev is not None:
             ev[0].record(stream)
-        mla.decode(q, kv, bt, sl, wl.scale, wl.causal, meta, out=out, lse=lse, workspace=ws, phase="split")
+        decode(q, kv, bt, sl, meta, out, lse, ws, "split")
         if ev is not None:
             ev[1].record(stream)
-        mla.decode(q, kv, bt, sl, wl.scale, wl.causal, meta, out=out, lse=lse, workspace=ws, phase="combine")
+        decode(q, kv, bt, sl, meta, out, lse, ws, "combine")
 
     for _ in range(args.warmup):
         step()
@@ -388,7 +416,44 @@ def main():
 
     # end to end through the host entry point: pinned host inputs in, host outputs out
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and fp8:
+        # the fp8 path has no host entry point: the same work through the Python API, each step
+        # copying the inputs from pinned host memory and the results back, then synchronising
+        qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
+        kvh = torch.from_numpy(inp["kv8"]).pin_memory()
+        bth = torch.from_numpy(inp["block_table"]).pin_memory()
+        slh = torch.from_numpy(inp["seqlens"]).pin_memory()
+        oh = torch.empty(tuple(out.shape), dtype=torch.bfloat16).pin_memory()
+        lh = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+        qd, kvd, btd, sld = torch.empty_like(q), torch.empty_like(kv), torch.empty_like(bt), torch.empty_like(sl)
+
+        def host_step():
+            for d, h in ((qd, qh), (kvd, kvh), (btd, bth), (sld, slh)):
+                d.copy_(h, non_blocking=True)
+            meta = mla.get_metadata(sld, wl.h_q, wl.s_q, num_parts=num_parts, fixed_cost=fixed_cost)
+            decode(qd, kvd, btd, sld, meta, out, lse, ws, "both")
+            oh.copy_(out, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+            stream.synchronize()
+
+        for _ in range(2):
+            host_step()
+        if dist is not None:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            host_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dev)[0]
+        h2d = sum(x.numel() * x.element_size() for x in (qh, kvh, bth, slh))
+        d2h = oh.numel() * 2 + lh.numel() * 4
+        e2e = {"value": bytes_all / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "Python API (decode_fp8) with pinned-host copies in and out, synchronised every step"}
+    elif args.e2e_steps > 0:
         hd = mla.HostDecoder(wl.batch, wl.s_q, wl.h_q, kv.shape[0], bt.shape[1], device=dev,
                              num_parts=num_parts, fixed_cost=fixed_cost)
         qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
@@ -427,15 +492,17 @@ def main():
         else:
             roof = {"bound": "tensor", "achieved": ach_tf, "peak": tfl_burst, "unit": "TFLOP/s",
                     "frac": ach_tf / tfl_burst}
-        roof.update({"traffic": profiled_traffic(), "kernel": "mla decode split kernel",
+        roof.update({"traffic": profiled_traffic(args.kv),
+                     "kernel": "mla decode split kernel" + (" (fp8 cache)" if fp8 else ""),
                      "peak_source": src + " (MEASURED_PEAKS.json)" if src == "measured" else "fallback",
                      "algorithmic_bytes_per_launch": counts["bytes"], "algorithmic_flops_per_launch": counts["flops"],
                      "launch_ms": split_avg_ms, "hbm_frac": ach_gbs / hbm, "tensor_frac": ach_tf / tfl_burst,
                      "tensor_frac_sustained": ach_tf / tfl_sust})
-        line = {"metric": METRIC, "value": value, "unit": "TB/s", "tflops": tflops, "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": describe(wl), "batch": wl.batch, "h_q": wl.h_q, "s_q": wl.s_q,
+        line = {"metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": "TB/s", "tflops": tflops,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f16 (fp8 E4M3 cache)" if fp8 else "bf16", "data": "synthetic",
+                "config": {"workload": describe(wl, args.kv), "kv": args.kv, "batch": wl.batch, "h_q": wl.h_q, "s_q": wl.s_q,
                            "causal": wl.causal, "num_parts": num_parts, "fixed_cost": fixed_cost,
                            "l2": ("inputs larger than L2 (KV cache %.0f MB > 126 MB); no flush" % (counts["kv_bytes"] / 1e6)
                                   if flush is None else "inputs (%.1f MB) fit in L2: a 256 MB write flushes L2 between "
@@ -446,7 +513,7 @@ def main():
                     "ms_per_step": graph_ms, "value": job_throughput(counts["bytes"], world, graph_ms), "unit": "TB/s",
                     "note": "the same step (metadata + split + combine) captured once in a CUDA graph and replayed"}}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, inp)
+            line["cpu_baseline"] = cpu_baseline(wl, inp, kv=args.kv)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

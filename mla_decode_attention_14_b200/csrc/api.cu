@@ -285,13 +285,16 @@ int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_bl
                              num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
                              workspace, workspace_bytes);
     if (rc != MLA_OK) return rc;
-    // kv_scale = mu 2^-k with mu in [1, 2): frexp gives kv_scale = f 2^e, f in [0.5, 1)
+    // kv_scale = mu 2^-k with mu in [1, 2): frexp gives kv_scale = f 2^e, f in [0.5, 1). The kernel's
+    // fp16 form of a latent byte is e4m3 * 2^-8, so the latent side carries mu 2^-8 = kv_scale 2^(k-8):
+    // the rotary query dims are multiplied by 2^(k-8) to match, the scores by 2^-(k-8), the output by
+    // kv_scale 2^8.
     if (!std::isfinite(kv_scale) || !(kv_scale > 0.f)) return MLA_ERR_INVALID_ARG;
     int e2 = 0;
     const float f = std::frexp(kv_scale, &e2);
     const int k = 1 - e2;
     if (k < -64 || k > 64) return MLA_ERR_INVALID_ARG;
-    const float sl2 = scale * 1.4426950408889634f * std::ldexp(1.f, -k);
+    const float sl2 = scale * 1.4426950408889634f * std::ldexp(1.f, 8 - k);
     if (!std::isfinite(sl2)) return MLA_ERR_INVALID_ARG;
     rc = check_device();
     if (rc != MLA_OK) return rc;
@@ -299,9 +302,9 @@ int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_bl
                                  num_splits, num_parts, batch, s_q, h_q, scale, causal, out, lse,
                                  workspace);
     p.scale_log2 = sl2;
-    p.v_scale = kv_scale;
+    p.v_scale = kv_scale * 256.f;
     p.q_lat_mul = 2.f * f;
-    p.q_rope_mul = std::ldexp(1.f, k);
+    p.q_rope_mul = std::ldexp(1.f, k - 8);
     CUtensorMap map_lat, map_rope;
     rc = cache_maps(kv_cache_fp8, num_blocks, 1, &map_lat, &map_rope);
     if (rc != MLA_OK) return rc;

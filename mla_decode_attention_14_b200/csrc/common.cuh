@@ -39,9 +39,10 @@ struct DecodeParams {
     int causal;
     float scale;                   // softmax scale
     float scale_log2;              // scale * log2(e) (fp8 cache: also times 2^-k, see q_rope_mul)
-    // fp8 cache only: a latent byte x stands for v_scale * e4m3(x), v_scale = q_lat_mul * 2^-k with
-    // q_lat_mul in [1, 2); the latent query dims are multiplied by q_lat_mul, the rotary ones by
-    // q_rope_mul = 2^k, and the output by v_scale.
+    // fp8 cache only: a latent byte x stands for kv_scale * e4m3(x), kv_scale = q_lat_mul * 2^-k with
+    // q_lat_mul in [1, 2), and the kernel's fp16 form of it is e4m3(x) * 2^-8; the latent query dims
+    // are multiplied by q_lat_mul, the rotary ones by q_rope_mul = 2^(k-8), the output by
+    // v_scale = kv_scale * 2^8.
     float v_scale, q_lat_mul, q_rope_mul;
 };
 

@@ -50,7 +50,6 @@
 //    kernel; whole sequences are written straight to bf16 out / fp32 lse.
 // Every wait is bounded; a timeout sets the device error word and the CTA exits cleanly.
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -60,31 +59,29 @@ using namespace sm100;
 
 namespace dec {
 constexpr int kStages = 5;
-constexpr int kFirstSoftWarp = 4;                 // warpgroup 0: TMA producer, Gemm1 issuer, (idle), Gemm2 issuer
 constexpr int kSoftWarps = 8;                     // two per SM sub-partition
-constexpr int kThreads = 32 * (kFirstSoftWarp + kSoftWarps);  // 384
+// bf16 cache: warpgroup 0 = TMA producer, Gemm1 issuer, (idle), Gemm2 issuer; softmax from warp 4.
+// fp8 cache: warpgroup 1 = four converter warps (one per SM sub-partition); softmax from warp 8.
+constexpr int kConvWarps = 4;
+template <bool F8> constexpr int first_soft_warp() { return F8 ? 4 + kConvWarps : 4; }
+template <bool F8> constexpr int num_threads() { return 32 * (first_soft_warp<F8>() + kSoftWarps); }  // 384 / 512
 constexpr int kTq = 2;                            // token halves per block
 constexpr int kTokPer = kBlk / kTq;               // 32 tokens per softmax thread
 // Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 = 64,512); warpgroup 0
 // drops to 96 and the two softmax warpgroups rise to 200: 128 x 96 + 256 x 200 = 63,488 <= 64,512.
-constexpr uint32_t kRegsControl = 96, kRegsSoftmax = 200;
+// fp8: 512 x 128 = 65,536 at launch; the control and converter warpgroups drop to 56:
+// 2 x 128 x 56 + 256 x 200 = 65,536.
+constexpr uint32_t kRegsControl = 96, kRegsSoftmax = 200, kRegsSmall = 56;
 constexpr int kBoxBytes = kBlk * 128;                      // 64 tokens x 64 bf16 (128-byte swizzle)
 constexpr int kRopeBoxBytes = kBlk * 64;                   // 64 tokens x 32 bf16 (64-byte swizzle)
 constexpr int kStageBytes = 4 * kBoxBytes + kRopeBoxBytes;  // 36,864: half of one cache block
-constexpr int kRingBytes = kStages * kStageBytes;          // shared memory of the KV ring
-// fp8 cache (640-byte token records: 512 E4M3 latent bytes, then 64 bf16 rotary dims): a 4-stage
-// ring of raw half-records (two 64-token x 128-byte latent boxes, 128-byte swizzle, and the rotary
-// box) and, behind it in the same shared memory, 3 buffers of the latent half converted to fp16 in
-// the bf16 stage's layout (four 64 x 64 boxes), which both GEMMs read.
-constexpr int kStages8 = 4, kConvBufs = 3;
-constexpr int kRawBoxBytes = kBlk * 128;                            // 64 tokens x 128 E4M3
-constexpr int kRawStageBytes = 2 * kRawBoxBytes + kRopeBoxBytes;    // 20,480
-constexpr int kConvBytes = 4 * kBoxBytes;                           // 32,768
-constexpr int kConvBase = kStages8 * kRawStageBytes;                // 81,920
-static_assert(kConvBase + kConvBufs * kConvBytes <= kRingBytes, "fp8 ring must fit the bf16 ring");
-template <bool F8> constexpr int ring_stages() { return F8 ? kStages8 : kStages; }
-template <bool F8> constexpr int stage_bytes() { return F8 ? kRawStageBytes : kStageBytes; }
-template <bool F8> constexpr int rope_offset() { return F8 ? 2 * kRawBoxBytes : 4 * kBoxBytes; }
+// fp8 cache (640-byte token records: 512 E4M3 latent bytes, then 64 bf16 rotary dims): the same
+// stages. TMA puts the two 64-token x 128-byte E4M3 latent boxes (128-byte swizzle) where fp16
+// boxes 2 and 3 go and the rotary box where it always goes; the converter warps then expand the
+// latent in place into the four fp16 boxes, so both GEMMs read the bf16 layout (in fp16).
+constexpr int kRawBoxBytes = kBlk * 128;                 // 64 tokens x 128 E4M3
+constexpr int kF8LoadBytes = 2 * kRawBoxBytes + kRopeBoxBytes;  // 20,480 loaded per stage
+constexpr int kRopeOffset = 4 * kBoxBytes;
 constexpr float kRescaleThreshold = 8.0f;                  // log2 units: rescale O when max grows > 2^8
 // The pair exchanges R = 2^((s - m) / 2 + 15), the square root of a factor, in fp16: R <= 2^15
 // (< 65504), normal (full 11-bit precision) while s - m >= -58 and subnormal down to -78, so the
@@ -104,13 +101,13 @@ constexpr int kXchgEBytes = 2 * kBlk * 128 * 2;    // two slots of 128 rows x 64
 constexpr int kXchgOffBytes = 2 * kTq * 128 * 4;   // two slots of 128 rows x 2 fp32 offsets
 
 struct __align__(1024) Smem {
-    uint8_t ring[kRingBytes];  // KV ring (bf16: kStages stages; fp8: raw stages, then fp16 buffers)
+    uint8_t stage[kStages][kStageBytes];  // KV ring
     uint4 xchg[(kXchgEBytes + kXchgOffBytes) / 16];  // peer factors R (fp16) [slot][token half][16 B][row]
                                                      // + row offsets (fp32) [slot][token half][row]
     float xmax[2][kTq][128];  // per-row exchange between the two token halves (block max bound; sums)
     uint8_t q_rope[128 * 64];             // rotary query dims [128 rows x 32], K-major, 64-byte swizzle
     uint64_t kv_full[kStages], kv_empty[kStages];
-    uint64_t conv_full[kConvBufs], conv_empty[kConvBufs];  // fp8 cache: converted latent buffers
+    uint64_t conv_full[kStages];  // fp8 cache: the stage's latent is in fp16
     uint64_t s_full, s_free, p_full, p_free, o_full, o_free, q_full, mma_done;
     uint64_t xfull[2];  // receive slots filled by the peer
     uint32_t tmem_base;
@@ -118,10 +115,6 @@ struct __align__(1024) Smem {
 };
 
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory (with 1 KB for alignment) must fit 227 KB");
-
-template <bool F8>
-__device__ __forceinline__ uint8_t *stage_ptr(Smem &sm, int s) { return sm.ring + s * stage_bytes<F8>(); }
-__device__ __forceinline__ uint8_t *conv_ptr(Smem &sm, int c) { return sm.ring + kConvBase + c * kConvBytes; }
 
 struct Piece {
     int seq, lo, hi, n, nsplit, slot;
@@ -192,14 +185,13 @@ struct BlockWalker {
 template <bool F8>
 __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map_lat, const CUtensorMap *map_rope,
                          const int32_t *meta, uint32_t half) {
-    constexpr int NS = ring_stages<F8>();
     const uint64_t policy = l2_evict_first_policy();
     BlockWalker w;
     w.init(meta, p);
     int gidx = 0;
     bool bad_block = false;
     for (; w.live; w.advance(p), ++gidx) {
-        const int s = gidx % NS, fill = gidx / NS;
+        const int s = gidx % kStages, fill = gidx / kStages;
         if (fill > 0 && !mbar_wait(&sm.kv_empty[s], (fill - 1) & 1, &sm.abort)) break;
         const int phys = w.blk < p.bt_stride ? __ldg(&p.block_table[(size_t)w.pc.seq * p.bt_stride + w.blk]) : -1;
         if (phys < 0 || (int64_t)phys >= p.num_blocks) {
@@ -207,26 +199,26 @@ __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map
             mbar_arrive(&sm.kv_full[s]);  // consumers run on stale data; the error word reports it
             continue;
         }
-        mbar_arrive_expect_tx(&sm.kv_full[s], stage_bytes<F8>());
+        mbar_arrive_expect_tx(&sm.kv_full[s], F8 ? kF8LoadBytes : kStageBytes);
         const int y = phys * kBlk;
-        uint8_t *dst = stage_ptr<F8>(sm, s);
+        uint8_t *dst = sm.stage[s];
         if constexpr (F8) {  // coordinates: bytes of the record (latent), bf16 elements (rotary)
 #pragma unroll
             for (int b = 0; b < 2; ++b)
-                tma_load_2d(dst + b * kRawBoxBytes, map_lat, 256 * (int)half + 128 * b, y, &sm.kv_full[s], policy);
-            tma_load_2d(dst + rope_offset<F8>(), map_rope, 256 + 32 * (int)half, y, &sm.kv_full[s], policy);
+                tma_load_2d(dst + (2 + b) * kBoxBytes, map_lat, 256 * (int)half + 128 * b, y, &sm.kv_full[s], policy);
+            tma_load_2d(dst + kRopeOffset, map_rope, 256 + 32 * (int)half, y, &sm.kv_full[s], policy);
         } else {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
                 tma_load_2d(dst + b * kBoxBytes, map_lat, 256 * (int)half + 64 * b, y, &sm.kv_full[s], policy);
-            tma_load_2d(dst + rope_offset<F8>(), map_rope, 512 + 32 * (int)half, y, &sm.kv_full[s], policy);
+            tma_load_2d(dst + kRopeOffset, map_rope, 512 + 32 * (int)half, y, &sm.kv_full[s], policy);
         }
     }
     if (bad_block) raise_error(kErrBounds);
     // every load still in flight must land before the CTA may exit
-    for (int k = max(0, gidx - NS); k < gidx; ++k) {
+    for (int k = max(0, gidx - kStages); k < gidx; ++k) {
         const long long t0 = clock64();
-        while (!mbar_sleep_test(&sm.kv_full[k % NS], (k / NS) & 1) && clock64() - t0 < kSpinCycles) {
+        while (!mbar_sleep_test(&sm.kv_full[k % kStages], (k / kStages) & 1) && clock64() - t0 < kSpinCycles) {
         }
     }
 }
@@ -253,53 +245,63 @@ __device__ void zero_tail_rows(uint8_t *st, int valid, int lane) {
     __syncwarp();
 }
 
-// fp8 cache, warp 2: the latent half of every block from E4M3 to fp16 -- exact, every E4M3 value is
-// an fp16 number -- into a buffer in the layout the MMA descriptors read (the bf16 stage's four
-// 128-byte-swizzled boxes of 64 tokens x 64 dims). Rows past a sequence's end are written as zeros,
-// so undefined tail contents never reach Gemm2. Lane mapping: each group of 8 lanes takes 16-byte
-// chunks 0-3 of one row of a row pair and chunks 4-7 of the other row, so the group's reads (one
-// chunk each) and writes (two chunks each) both fall on 8 distinct 16-byte bank groups.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// fp8 cache, warps 4-7: the latent half of every block from E4M3 to fp16 bit patterns, in place,
+// into the layout the MMA descriptors read (the bf16 stage's four 128-byte-swizzled boxes of 64
+// tokens x 64 dims). Raw box 0 (in fp16 box 2's place) becomes boxes 0-1; after a barrier of the four
+// warps, raw box 1 (in box 3's place) becomes boxes 2-3: every row of box 3 is written by the
+// instruction that read the same row of raw box 1, so the expansion never overwrites unread bytes.
+// The E4M3 byte s.eeee.mmm placed as the fp16 pattern s.0eeee.mmm0000000 is the fp16 number
+// e4m3 * 2^-8 -- exactly, subnormals included (both formats put the subnormal point at exponent
+// field 0) -- so the conversion is four integer operations per pair of values (byte permute, mask,
+// shift, merge); the 2^-8 is folded into the score and output scales. (The hardware e4m3x2 -> f16x2
+// conversion took ~8k cycles per block on one warp.) Rows past a sequence's end are written as
+// zeros, so undefined tail contents never reach Gemm2. Lane mapping: each group of 8 lanes takes
+// 16-byte chunks 0-3 of one row of a row pair and chunks 4-7 of the other row, so the group's reads
+// (one chunk each) and writes (two chunks each) fall on 8 distinct bank groups.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
+    const uint32_t t = __byte_perm(w, 0u, sel);  // the two bytes at bits 8-15 and 24-31
+    return (t & 0x80008000u) | ((t & 0x7f007f00u) >> 1);
 }
 
+constexpr int kConvBarrier = 5;  // named barrier of the four converter warps (1-4: softmax row pairs)
+
 __device__ void convert_warp(Smem &sm, const DecodeParams &p, const int32_t *meta) {
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) & (kConvWarps - 1);
     const int u = lane & 7, hp = (lane >> 3) & 1, pq = lane >> 4;  // chunk, half of the pair, pair of the step
     const int k0 = 2 * (u & 3);                                     // first fp16 chunk of the box row
     volatile int *abort = &sm.abort;
     BlockWalker w;
     w.init(meta, p);
     for (int g = 0; w.live; w.advance(p), ++g) {
-        const int s = g % kStages8, c = g % kConvBufs;
-        if (!warp_wait(&sm.kv_full[s], (g / kStages8) & 1, abort, lane)) break;
-        if (g >= kConvBufs && !warp_wait(&sm.conv_empty[c], (g / kConvBufs - 1) & 1, abort, lane)) break;
+        const int s = g % kStages;
+        if (!warp_wait(&sm.kv_full[s], (g / kStages) & 1, abort, lane)) break;
         const int valid = w.tail() ? w.pc.n - w.blk * kBlk : kBlk;
-        const uint8_t *raw = stage_ptr<true>(sm, s);
-        uint8_t *dst = conv_ptr(sm, c);
-#pragma unroll 4
-        for (int it = 0; it < 32; ++it) {
-            const int pi = 2 * it + pq;  // row pair over both raw boxes: 2 x 32 pairs
-            const int bx = pi >> 5, row = 2 * (pi & 31) + ((u >> 2) ^ hp), sw = row & 7;
-            uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-            if (row < valid) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(raw + bx * kRawBoxBytes + row * 128 + ((u ^ sw) << 4));
-                lo = make_uint4(e4m3x2_to_f16x2(x.x & 0xffffu), e4m3x2_to_f16x2(x.x >> 16),
-                                e4m3x2_to_f16x2(x.y & 0xffffu), e4m3x2_to_f16x2(x.y >> 16));
-                hi = make_uint4(e4m3x2_to_f16x2(x.z & 0xffffu), e4m3x2_to_f16x2(x.z >> 16),
-                                e4m3x2_to_f16x2(x.w & 0xffffu), e4m3x2_to_f16x2(x.w >> 16));
+        uint8_t *dst = sm.stage[s];
+#pragma unroll 1
+        for (int bx = 0; bx < 2; ++bx) {  // raw box bx: 32 row pairs, 4 steps of 2 pairs per warp
+            if (bx == 1) named_bar_sync(kConvBarrier, 32 * kConvWarps);  // raw box 0 read by all four warps
+#pragma unroll
+            for (int it = 16 * bx + cw; it < 16 * bx + 16; it += kConvWarps) {
+                const int pi = 2 * it + pq;  // row pair over both raw boxes: 2 x 32 pairs
+                const int row = 2 * (pi & 31) + ((u >> 2) ^ hp), sw = row & 7;
+                uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+                if (row < valid) {
+                    const uint4 x =
+                        *reinterpret_cast<const uint4 *>(dst + (2 + bx) * kBoxBytes + row * 128 + ((u ^ sw) << 4));
+                    // bytes 0,1 -> word 0; bytes 2,3 -> word 1 (little-endian: the lower dim in the low half)
+                    lo = make_uint4(e4m3x2_to_f16x2_scaled(x.x, 0x1404u), e4m3x2_to_f16x2_scaled(x.x, 0x3424u),
+                                    e4m3x2_to_f16x2_scaled(x.y, 0x1404u), e4m3x2_to_f16x2_scaled(x.y, 0x3424u));
+                    hi = make_uint4(e4m3x2_to_f16x2_scaled(x.z, 0x1404u), e4m3x2_to_f16x2_scaled(x.z, 0x3424u),
+                                    e4m3x2_to_f16x2_scaled(x.w, 0x1404u), e4m3x2_to_f16x2_scaled(x.w, 0x3424u));
+                }
+                uint8_t *o = dst + (2 * bx + (u >> 2)) * kBoxBytes + row * 128;
+                *reinterpret_cast<uint4 *>(o + ((k0 ^ sw) << 4)) = lo;
+                *reinterpret_cast<uint4 *>(o + (((k0 + 1) ^ sw) << 4)) = hi;
             }
-            uint8_t *o = dst + (2 * bx + (u >> 2)) * kBoxBytes + row * 128;
-            *reinterpret_cast<uint4 *>(o + ((k0 ^ sw) << 4)) = lo;
-            *reinterpret_cast<uint4 *>(o + (((k0 + 1) ^ sw) << 4)) = hi;
         }
         fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&sm.conv_full[c]);
-            mbar_arrive(&sm.kv_empty[s]);  // the raw latent is consumed (Gemm1 still reads the rotary box)
-        }
+        if (lane == 0) mbar_arrive(&sm.conv_full[s]);  // one arrival per converter warp
     }
 }
 
@@ -314,23 +316,20 @@ template <bool F8>
 __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
     constexpr uint32_t id1 = idesc_bf16_f32(128, 64, 0);  // S = Q K^T: K-major B
     constexpr uint32_t id1_lat = F8 ? idesc_f16_f32(128, 64, 0) : id1;
-    constexpr int NS = ring_stages<F8>();
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
     BlockWalker w;
     w.init(meta, p);
     for (int g = 0; w.live; w.advance(p), ++g) {
         if (w.first() && !warp_wait(&sm.q_full, w.piece_k & 1, abort, lane)) break;
-        const int s = g % NS, cb = g % kConvBufs;
-        if (!warp_wait(&sm.kv_full[s], (g / NS) & 1, abort, lane)) break;
-        if (F8 && !warp_wait(&sm.conv_full[cb], (g / kConvBufs) & 1, abort, lane)) break;
+        const int s = g % kStages;
+        if (!warp_wait(F8 ? &sm.conv_full[s] : &sm.kv_full[s], (g / kStages) & 1, abort, lane)) break;
         if (g > 0 && !warp_wait(&sm.s_free, (g - 1) & 1, abort, lane)) break;
         if (lane == 0) {
             tc_fence_after();
             // descriptors: one base each, then constant offsets (address field is in 16-byte units)
-            const uint8_t *lat = F8 ? conv_ptr(sm, cb) : stage_ptr<F8>(sm, s);
-            const uint64_t kd = smem_desc(smem_addr(lat), 16, 1024, 2);
-            const uint64_t rd = smem_desc(smem_addr(stage_ptr<F8>(sm, s)) + rope_offset<F8>(), 16, 512, 4);
+            const uint64_t kd = smem_desc(smem_addr(sm.stage[s]), 16, 1024, 2);
+            const uint64_t rd = smem_desc(smem_addr(sm.stage[s]) + kRopeOffset, 16, 512, 4);
             const uint64_t qd = smem_desc(smem_addr(sm.q_rope), 16, 512, 4);
 #pragma unroll
             for (int k = 0; k < 16; ++k)  // latent k-steps, A (Q) from TMEM
@@ -340,7 +339,6 @@ __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
             for (int c = 0; c < 2; ++c)  // rotary k-steps, A from shared memory
                 mma_ss(tmem + kTmemS, qd + 2 * c, rd + 2 * c, id1, 1u);
             mma_commit(&sm.s_full);
-            if (F8) mma_commit(&sm.kv_empty[s]);  // the raw stage's rotary box is consumed
         }
         __syncwarp();
     }
@@ -351,7 +349,7 @@ __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
 template <bool F8>
 __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
     constexpr uint32_t id2 = F8 ? idesc_f16_f32(128, 256, 1) : idesc_bf16_f32(128, 256, 1);  // MN-major B
-    constexpr int NS = ring_stages<F8>(), kTerms = F8 ? 1 : 2;
+    constexpr int kTerms = F8 ? 1 : 2;
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
     BlockWalker w;
@@ -359,13 +357,13 @@ __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
     for (int g = 0; w.live; w.advance(p), ++g) {
         if (!warp_wait(&sm.p_full, g & 1, abort, lane)) break;
         if (w.first() && w.piece_k > 0 && !warp_wait(&sm.o_free, (w.piece_k - 1) & 1, abort, lane)) break;
-        const int s = g % NS, cb = g % kConvBufs;
+        const int s = g % kStages;
         // P of block g exists, so Gemm1 of block g has completed and its tile may be edited (the fp8
         // path's converter has already zeroed the tail rows)
-        if (!F8 && w.tail()) zero_tail_rows(stage_ptr<F8>(sm, s), w.pc.n - w.blk * kBlk, lane);
+        if (!F8 && w.tail()) zero_tail_rows(sm.stage[s], w.pc.n - w.blk * kBlk, lane);
         if (lane == 0) {
             tc_fence_after();
-            const uint64_t vd = smem_desc(smem_addr(F8 ? conv_ptr(sm, cb) : stage_ptr<F8>(sm, s)), 4 * 2048, 1024, 2);
+            const uint64_t vd = smem_desc(smem_addr(sm.stage[s]), 4 * 2048, 1024, 2);
             const bool first = w.first();
 #pragma unroll
             for (int hl = 0; hl < kTerms; ++hl)  // P_hi, then P_lo, A from TMEM
@@ -374,7 +372,7 @@ __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
                     mma_ts(tmem + kTmemO, tmem + (hl ? kTmemPlo : kTmemPhi) + 8 * kk, vd + 128 * kk, id2,
                            (!first || hl > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&sm.p_free);
-            mma_commit(F8 ? &sm.conv_empty[cb] : &sm.kv_empty[s]);
+            mma_commit(&sm.kv_empty[s]);
             if (w.last()) mma_commit(&sm.o_full);
         }
         __syncwarp();
@@ -421,8 +419,8 @@ __device__ __forceinline__ uint32_t bf16x2_pow2(uint32_t v, float pow2, bool &ba
 // Q of piece `pc`: latent half -> TMEM (this warp's lanes, its 64 of the 128 columns),
 // rotary half -> shared memory (its 2 of the 4 16-byte chunks of the row).
 // fp8 cache, with the latent scale written as mu 2^-k (mu in [1, 2)): the latent dims go to TMEM
-// as fp16(q mu) and the rotary dims as q 2^k (exact), so that the accumulated score is 2^k times
-// scale^-1 s; the kernel's score scale carries the 2^-k.
+// as fp16(q mu) and the rotary dims as q 2^(k-8) (exact), matching the converted cache's e4m3 2^-8,
+// so that the accumulated score is 2^(k-8) times s / scale; the kernel's score scale carries 2^-(k-8).
 template <bool F8>
 __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &pc) {
     if (c.warp_ok) {
@@ -537,7 +535,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     c.half = half;
     const int warp = threadIdx.x >> 5;
     const int wq = warp & 3;
-    c.th = (warp - kFirstSoftWarp) >> 2;
+    c.th = (warp - first_soft_warp<F8>()) >> 2;
     c.lane = threadIdx.x & 31;
     c.i = wq * 32 + c.lane;  // row within the group == TMEM lane
     c.lane_off = (uint32_t)(wq * 32) << 16;
@@ -595,7 +593,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         }
         // peer factors of block g (slot g % 2)
         const int slot = g & 1;
-        if (threadIdx.x == 32 * kFirstSoftWarp) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
+        if (threadIdx.x == 32 * first_soft_warp<F8>()) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
         if (!mbar_wait_cluster(&sm.xfull[slot], (g >> 1) & 1, abort)) return;
         const float m_peer = c.warp_ok ? xo[(slot * kTq + c.th) * 128 + c.i] : -INFINITY;
         const float mbu_half = m_own + m_peer;
@@ -813,7 +811,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
 }
 
 template <bool F8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(num_threads<F8>(), 1)
 decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_rope,
                     const DecodeParams p, const int groups) {
     extern __shared__ uint8_t smem_raw[];
@@ -828,11 +826,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], F8 ? 2 : 1);  // fp8: the converter and Gemm1's commit
-        }
-        for (int b = 0; b < kConvBufs; ++b) {
-            mbar_init(&sm.conv_full[b], 1);
-            mbar_init(&sm.conv_empty[b], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.conv_full[s], kConvWarps);
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.s_free, kSoftWarps);
@@ -857,8 +852,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     cluster_sync();  // the peer's barriers exist before any exchange targets them
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp < kFirstSoftWarp) {
-        setmaxnreg_dec<kRegsControl>();
+    if (F8 && warp >= 4 && warp < first_soft_warp<F8>()) {
+        setmaxnreg_dec<kRegsSmall>();
+        convert_warp(sm, p, meta);
+    } else if (warp < 4) {
+        setmaxnreg_dec<F8 ? kRegsSmall : kRegsControl>();
         if (warp == 0) {
             if (lane == 0) producer<F8>(sm, p, &map_lat, &map_rope, meta, half);
         } else {
@@ -868,8 +866,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
             } else if (warp == 1) {
                 gemm1_warp<F8>(sm, p, meta, tmem);
                 drain_mmas(sm);
-            } else if (F8) {
-                convert_warp(sm, p, meta);
             }
         }
     } else {
@@ -896,11 +892,20 @@ cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_la
     const int groups = (p.rows + 127) / 128;
     const size_t smem = decode_sm100_smem_bytes();
     auto kernel = fp8 ? dec::decode_sm100_kernel<true> : dec::decode_sm100_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int threads = fp8 ? dec::num_threads<true>() : dec::num_threads<false>();
+    // setmaxnreg redistributes the registers the block was launched with: the warpgroups' shares must
+    // fit in what the compiler gave the kernel, or the raising warps would wait forever
+    const int need = fp8 ? 2 * 128 * (int)dec::kRegsSmall + 256 * (int)dec::kRegsSoftmax
+                         : 128 * (int)dec::kRegsControl + 256 * (int)dec::kRegsSoftmax;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * threads < need) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * p.num_parts * groups, 1, 1);
-    cfg.blockDim = dim3(dec::kThreads, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

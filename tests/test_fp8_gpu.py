@@ -138,6 +138,20 @@ def test_single_token_sequences_return_dequantized_rows():
         assert torch.equal(out[i, 0].cpu(), want.expand(128, 512))
 
 
+def test_subnormal_codes_are_not_flushed():
+    """Every latent byte an E4M3 subnormal (exponent field 0): the kernel's fp16 form of those is
+    subnormal too, and the tensor core must keep them. A latent scale of 2^6 makes the values
+    ~0.1-0.9, so a flush to zero would show as a wrong output."""
+    wl = W.custom(2, 64, 1, [200, 70])
+    inp = W.make_inputs_fp8(wl, seed=12, tail="nan", kv_scale=2.0 ** 6)
+    rng = np.random.default_rng(3)
+    lat = inp["kv8"][..., :512]
+    codes = rng.integers(1, 8, size=lat.shape).astype(np.uint8) | (rng.integers(0, 2, size=lat.shape).astype(np.uint8) << 7)
+    nan_rows = lat == W.F8_NAN
+    lat[...] = np.where(nan_rows, lat, codes)
+    full_parity_fp8(inp, num_parts=3, what="subnormal codes")
+
+
 def test_empty_sequences_give_zero_and_neg_inf():
     wl = W.custom(3, 16, 2, [0, 70, 1], causal=True)
     inp = W.make_inputs_fp8(wl, seed=6)
