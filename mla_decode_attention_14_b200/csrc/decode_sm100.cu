@@ -615,8 +615,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
 #pragma unroll
             for (int j = 0; j < kTokPer; j += 2) {
                 const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
-                e_own[j] *= e2.x;
-                e_own[j + 1] *= e2.y;
+                unpack2(mul2(pack2(e_own[j], e_own[j + 1]), pack2(e2.x, e2.y)), e_own[j], e_own[j + 1]);
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) t[j] = fmaxf(e_own[j], e_own[j + 16]);
@@ -686,8 +685,12 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         const int nslot = (g + 1) & 1;
         const uint32_t xbase = xchg_peer + (uint32_t)(((nslot * kTq + c.th) * 4) * 128 + c.i) * 16;
         const uint32_t xbar = xfull_peer0 + nslot * 8;
+        // The arithmetic runs on token pairs with the packed f32x2 instructions (two fp32 lanes per
+        // instruction, each rounded as its scalar form would be).
         uint32_t pk[kTokPer / 2], pl[kTokPer / 2];
-        float su[4] = {0.f, 0.f, 0.f, 0.f};
+        f32x2 su[4] = {0ull, 0ull, 0ull, 0ull};  // two lanes of partial row sums each (0 is +0, +0)
+        const f32x2 ff = pack2(f, f), hsl2 = pack2(0.5f * sl2, 0.5f * sl2), offnx = pack2(off_nx, off_nx);
+        const f32x2 minus1 = pack2(-1.f, -1.f);
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t wv[4];
@@ -695,23 +698,33 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
             for (int q = 0; q < 4; ++q) {
                 const int j = 8 * c4 + 2 * q;
                 // R of block g+1: 2^((s * scale_log2 - m) / 2 + 15), in [0, 2^15], 0 for masked tokens
-                snx[j] = ex2_approx(fmaf(snx[j], 0.5f * sl2, off_nx));
-                snx[j + 1] = ex2_approx(fmaf(snx[j + 1], 0.5f * sl2, off_nx));
+                float x0, x1;
+                unpack2(fma2(pack2(snx[j], snx[j + 1]), hsl2, offnx), x0, x1);
+                snx[j] = ex2_approx(x0);
+                snx[j + 1] = ex2_approx(x1);
                 __half2 two = __floats2half2_rn(snx[j], snx[j + 1]);
                 wv[q] = *reinterpret_cast<uint32_t *>(&two);
                 // P of block g
                 if constexpr (F8) {  // e_own holds t = R_own R_peer; P in fp16 (round to nearest)
-                    const float p0 = e_own[j] * e_own[j] * f, p1 = e_own[j + 1] * e_own[j + 1] * f;
-                    su[q] += p0 + p1;
+                    const f32x2 t = pack2(e_own[j], e_own[j + 1]);
+                    const f32x2 pp = mul2(mul2(t, t), ff);
+                    su[q] = add2(su[q], pp);
+                    float p0, p1;
+                    unpack2(pp, p0, p1);
                     __half2 ph = __floats2half2_rn(p0, p1);
                     pk[j >> 1] = *reinterpret_cast<uint32_t *>(&ph);
                 } else {
                     const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
-                    const float t0 = e_own[j] * e2.x, t1 = e_own[j + 1] * e2.y;
-                    const float p0 = t0 * t0 * f, p1 = t1 * t1 * f;
-                    su[q] += p0 + p1;
+                    const f32x2 t = mul2(pack2(e_own[j], e_own[j + 1]), pack2(e2.x, e2.y));
+                    const f32x2 pp = mul2(mul2(t, t), ff);
+                    su[q] = add2(su[q], pp);
+                    float p0, p1;
+                    unpack2(pp, p0, p1);
                     const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-                    const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u), r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                    // lo = P - hi, exact (hi is P with its low 16 bits cleared)
+                    float r0, r1;
+                    unpack2(fma2(pack2(__uint_as_float(u0 & 0xffff0000u), __uint_as_float(u1 & 0xffff0000u)), minus1, pp),
+                            r0, r1);
                     pk[j >> 1] = __byte_perm(u0, u1, 0x7632);
                     pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
                 }
@@ -721,7 +734,11 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         if (send)  // the row offset travels in the offsets area of the same slot
             st_async_b32(xchg_peer + (uint32_t)kXchgEBytes + (uint32_t)((nslot * kTq + c.th) * 128 + c.i) * 4,
                          __float_as_uint(m_nx), xbar);
-        l += (su[0] + su[1]) + (su[2] + su[3]);
+        {
+            float a0, a1;
+            unpack2(add2(add2(su[0], su[1]), add2(su[2], su[3])), a0, a1);
+            l += a0 + a1;
+        }
         // the P tile and O are free once Gemm2 of block g-1 has completed
         if (g > 0 && !mbar_wait(&sm.p_free, (g - 1) & 1, abort)) return;
         tc_fence_after();
