@@ -611,20 +611,14 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 ep[4 * c4 + 2] = v.z;
                 ep[4 * c4 + 3] = v.w;
             }
-            float t[16];
 #pragma unroll
             for (int j = 0; j < kTokPer; j += 2) {
                 const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
                 unpack2(mul2(pack2(e_own[j], e_own[j + 1]), pack2(e2.x, e2.y)), e_own[j], e_own[j + 1]);
             }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) t[j] = fmaxf(e_own[j], e_own[j + 16]);
-#pragma unroll
-            for (int k = 8; k >= 1; k >>= 1)
-#pragma unroll
-                for (int j = 0; j < k; ++j) t[j] = fmaxf(t[j], t[j + k]);
+            const float tmax = max32(e_own);
             const float mx_half =
-                (t[0] > 0.f && mbu_half != -INFINITY) ? 2.f * (__log2f(t[0]) - 2.f * kXScaleLog2) + mbu_half : -INFINITY;
+                (tmax > 0.f && mbu_half != -INFINITY) ? 2.f * (__log2f(tmax) - 2.f * kXScaleLog2) + mbu_half : -INFINITY;
             sm.xmax[g & 1][c.th][c.i] = mx_half;
             named_bar_sync(bar_id, 64);
             mbu = fmaxf(mx_half, sm.xmax[g & 1][c.th ^ 1][c.i]);
@@ -670,15 +664,9 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 4.f * kXScaleLog2);
         float m_nx, off_nx;
         {
-            float t[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) t[j] = fmaxf(snx[j], snx[j + 16]);
-#pragma unroll
-            for (int k = 8; k >= 1; k >>= 1)
-#pragma unroll
-                for (int j = 0; j < k; ++j) t[j] = fmaxf(t[j], t[j + k]);
-            const bool nx_none = t[0] == -INFINITY;
-            m_nx = nx_none ? -INFINITY : t[0] * sl2;  // sl2 > 0, so the max commutes with the scaling
+            const float smax = max32(snx);
+            const bool nx_none = smax == -INFINITY;
+            m_nx = nx_none ? -INFINITY : smax * sl2;  // sl2 > 0, so the max commutes with the scaling
             off_nx = nx_none ? 0.f : kXScaleLog2 - 0.5f * m_nx;
         }
         const bool send = nx_live && c.warp_ok;

@@ -279,6 +279,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// max of three fp32 values in one instruction (sm_100); -inf is the identity.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// max of 32 values in 17 instructions (three-input maxes, depth 4).
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+    float a[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) a[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    a[10] = fmaxf(v[30], v[31]);
+    const float b0 = fmax3(a[0], a[1], a[2]), b1 = fmax3(a[3], a[4], a[5]), b2 = fmax3(a[6], a[7], a[8]);
+    return fmax3(b0, b1, fmax3(b2, a[9], a[10]));
+}
+
 // Two fp32 lanes in one 64-bit register pair, for the packed f32x2 arithmetic of sm_100: one
 // instruction does two independent fp32 multiplies / adds / FMAs (each rounded to nearest).
 typedef unsigned long long f32x2;
