@@ -60,6 +60,13 @@ def _load():
         lib.oracle_decode_fp8.restype = ctypes.c_int
         lib.oracle_e4m3_decode.argtypes = [P, ctypes.c_int64, P]
         lib.oracle_e4m3_decode.restype = None
+        lib.oracle_e4m3_encode.argtypes = [P, ctypes.c_int64, P]
+        lib.oracle_e4m3_encode.restype = None
+        lib.oracle_append.argtypes = [P, ctypes.c_int, P, ctypes.c_int64, P, ctypes.c_int64, P, ctypes.c_int]
+        lib.oracle_append.restype = ctypes.c_int
+        lib.oracle_append_fp8.argtypes = [P, ctypes.c_int, P, ctypes.c_float, ctypes.c_int64, P, ctypes.c_int64, P,
+                                          ctypes.c_int]
+        lib.oracle_append_fp8.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -156,3 +163,40 @@ def e4m3_decode(codes) -> np.ndarray:
     out = np.empty(x.shape, dtype=np.float64)
     _load().oracle_e4m3_decode(_ptr(x), x.size, _ptr(out))
     return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """float32 -> OCP E4M3 codes, round to nearest even, saturating to +-448."""
+    v = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def append(new_kv_bits, kv_bits, block_table, seqlens):
+    """Write the new tokens ``new_kv_bits`` (uint16 bf16 ``[b, n_new, 576]``) into a copy of the bf16
+    cache at positions ``seqlens[b] + t``; returns the new cache."""
+    nk = np.ascontiguousarray(new_kv_bits, dtype=np.uint16)
+    kv = np.array(kv_bits, dtype=np.uint16, copy=True, order="C")
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    rc = _load().oracle_append(_ptr(nk), nk.shape[1], _ptr(kv), kv.shape[0], _ptr(bt), bt.shape[1], _ptr(sl),
+                               nk.shape[0])
+    if rc != 0:
+        raise ValueError("oracle_append: a row lands outside the table or the cache")
+    return kv
+
+
+def append_fp8(new_kv_bits, kv8, inv_scale: float, block_table, seqlens):
+    """The same into a copy of the fp8 cache: latent values times ``inv_scale`` (fp32) rounded to
+    E4M3, rotary dims copied; returns the new cache."""
+    nk = np.ascontiguousarray(new_kv_bits, dtype=np.uint16)
+    kv = np.array(kv8, dtype=np.uint8, copy=True, order="C")
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    rc = _load().oracle_append_fp8(_ptr(nk), nk.shape[1], _ptr(kv), float(np.float32(inv_scale)), kv.shape[0],
+                                   _ptr(bt), bt.shape[1], _ptr(sl), nk.shape[0])
+    if rc != 0:
+        raise ValueError("oracle_append_fp8: a row lands outside the table or the cache")
+    return kv
+

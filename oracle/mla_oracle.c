@@ -362,3 +362,94 @@ int oracle_decode_fp8(const uint16_t *q, const uint8_t *kv8, double kv_scale, in
 void oracle_e4m3_decode(const uint8_t *x, int64_t n, double *out) {
     for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_double(x[i]);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Appending new tokens to the paged cache (the step that precedes decode).     */
+/*                                                                            */
+/* Token t of sequence b's new tokens goes to position p = seqlens[b] + t of   */
+/* the sequence: cache row block_table[b][p / 64] * 64 + p % 64. bf16 cache:   */
+/* the 576 bf16 values are copied. fp8 cache: each latent value x (bf16,      */
+/* exactly a float) is multiplied by inv_scale in fp32 and written as the E4M3 */
+/* code of the product, rounded to nearest (ties to even) and saturated to    */
+/* +-448 (infinities too); NaN stays NaN; the rotary dims are copied as bf16.  */
+/* Returns 0, or -1 when a row would land outside the table or the cache.      */
+/* ------------------------------------------------------------------------- */
+
+/* fp32 -> E4M3 code, round to nearest even, saturating (OCP OFP8 E4M3, see e4m3_to_double). */
+static uint8_t e4m3_from_float(float v) {
+    uint32_t u;
+    memcpy(&u, &v, sizeof u);
+    const uint8_t sign = (uint8_t)((u >> 31) << 7);
+    if (isnan(v)) return (uint8_t)(sign | 0x7F);
+    double a = fabs((double)v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    /* the spacing of E4M3 values around a: 2^-9 below 2^-6 (subnormals), else 2^(e - 3) */
+    int e;
+    frexp(a, &e);          /* a = f * 2^e, f in [0.5, 1): the leading bit is 2^(e-1) */
+    int lead = e - 1;      /* a in [2^lead, 2^(lead+1)) */
+    if (lead < -6) lead = -6;
+    const double quantum = ldexp(1.0, lead - 3);
+    double q = a / quantum; /* exact: a power-of-two scaling */
+    double fl = floor(q), rem = q - fl;
+    if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0)) fl += 1.0;
+    const double r = fl * quantum; /* the rounded magnitude; may step up to the next binade */
+    if (r >= 448.0) return (uint8_t)(sign | 0x7E);
+    if (r == 0.0) return sign;
+    int re;
+    frexp(r, &re);
+    int rlead = re - 1;
+    if (rlead < -6) { /* subnormal: r = m * 2^-9 */
+        const int m = (int)(r / ldexp(1.0, -9));
+        return (uint8_t)(sign | m);
+    }
+    const int E = rlead + 7;
+    const int m = (int)((r / ldexp(1.0, rlead) - 1.0) * 8.0);
+    return (uint8_t)(sign | (E << 3) | m);
+}
+
+void oracle_e4m3_encode(const float *x, int64_t n, uint8_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_from_float(x[i]);
+}
+
+static int append_rows(const uint16_t *new_kv, int n_new, uint16_t *kv, uint8_t *kv8, float inv_scale,
+                       int64_t num_blocks, const int32_t *block_table, int64_t bt_stride,
+                       const int32_t *seqlens, int batch) {
+    if (!new_kv || (!kv && !kv8) || !block_table || !seqlens || n_new < 0 || batch < 0) return -1;
+    for (int b = 0; b < batch; ++b) {
+        for (int t = 0; t < n_new; ++t) {
+            const int64_t pos = (int64_t)(seqlens[b] > 0 ? seqlens[b] : 0) + t;
+            if (pos / OR_BLK >= bt_stride) return -1;
+            const int32_t phys = block_table[(size_t)b * bt_stride + pos / OR_BLK];
+            if (phys < 0 || phys >= num_blocks) return -1;
+            const int64_t row = (int64_t)phys * OR_BLK + pos % OR_BLK;
+            const uint16_t *src = new_kv + ((size_t)b * n_new + t) * OR_D_QK;
+            if (kv) {
+                memcpy(kv + (size_t)row * OR_D_QK, src, OR_D_QK * sizeof(uint16_t));
+            } else {
+                uint8_t *dst = kv8 + (size_t)row * OR_F8_REC;
+                for (int d = 0; d < OR_D_V; ++d) {
+                    const float x = (float)bf16_bits_to_double(src[d]);
+                    dst[d] = e4m3_from_float(x * inv_scale); /* one fp32 multiply, then the rounding */
+                }
+                for (int d = OR_D_V; d < OR_D_QK; ++d) {
+                    dst[OR_D_V + 2 * (d - OR_D_V)] = (uint8_t)(src[d] & 0xFF);
+                    dst[OR_D_V + 2 * (d - OR_D_V) + 1] = (uint8_t)(src[d] >> 8);
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+int oracle_append(const uint16_t *new_kv, int n_new, uint16_t *kv_cache, int64_t num_blocks,
+                  const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens, int batch) {
+    if (!kv_cache) return -1;
+    return append_rows(new_kv, n_new, kv_cache, NULL, 0.f, num_blocks, block_table, bt_stride, seqlens, batch);
+}
+
+int oracle_append_fp8(const uint16_t *new_kv, int n_new, uint8_t *kv8, float inv_scale, int64_t num_blocks,
+                      const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens, int batch) {
+    if (!kv8) return -1;
+    return append_rows(new_kv, n_new, NULL, kv8, inv_scale, num_blocks, block_table, bt_stride, seqlens, batch);
+}
+

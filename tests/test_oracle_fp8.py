@@ -137,3 +137,79 @@ def test_nan_tail_is_never_read():
     rb = oracle.decode_fp8(b["q"], b["kv8"], b["kv_scale"], b["block_table"], b["seqlens"], wl.scale, False)
     assert np.all(np.isfinite(ra[0]))
     assert np.array_equal(ra[0], rb[0]) and np.array_equal(ra[1], rb[1])
+
+
+# ---------------------------------------------------------------- E4M3 encoding and appends
+def test_e4m3_encoding_round_trips_every_finite_code():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle.e4m3_decode(codes).astype(np.float32)
+    fin = ~np.isnan(vals)
+    assert np.array_equal(oracle.e4m3_encode(vals)[fin], codes[fin])
+
+
+@pytest.mark.parametrize("x,code", [
+    (1.0625, 0x38),        # tie between 1 (mantissa 0) and 1.125 (1): to even, 1
+    (1.1875, 0x3A),        # tie between 1.125 (1) and 1.25 (2): to even, 1.25
+    (2.0 ** -10, 0x00),    # tie between 0 and the smallest subnormal 2^-9: to even, 0
+    (3 * 2.0 ** -10, 0x02),  # tie between 2^-9 (1) and 2^-8 (2): to even, 2
+    (-3 * 2.0 ** -10, 0x82),
+    (0.9999, 0x38),        # rounds up into the next binade
+    (460.0, 0x7E), (500.0, 0x7E), (float("inf"), 0x7E), (-1000.0, 0xFE),  # saturation to +-448
+    (float("nan"), 0x7F),
+])
+def test_e4m3_encoding_hand_worked_cases(x, code):
+    assert int(oracle.e4m3_encode(np.array([x], dtype=np.float32))[0]) == code
+
+
+def test_e4m3_encoding_matches_torch_in_range():
+    x = np.random.default_rng(0).standard_normal(100000).astype(np.float32) * 60
+    x = np.clip(x, -448, 448)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(x), ref)
+
+
+def _append_case(kv="bf16"):
+    wl = W.custom(3, 4, 1, [5, 64, 130])
+    gen = W.make_inputs_fp8 if kv == "fp8" else W.make_inputs
+    inp = gen(wl, seed=13, tail="normal", spare_blocks=2)
+    # the table must hold the new positions: lengths 5 + 3 stay in block 0, 64 + 3 spills into a new
+    # block, 130 + 3 stays in block 2; give sequence 1 a spare physical block for its second entry
+    bt = inp["block_table"].copy()
+    if bt.shape[1] < 3:
+        bt = np.concatenate([bt, np.full((3, 3 - bt.shape[1]), -1, np.int32)], axis=1)
+    free = sorted(set(range(inp["num_blocks"])) - set(int(v) for v in bt[bt >= 0]))
+    bt[1, 1] = free[0]
+    new = W.f32_to_bf16_bits(np.random.default_rng(1).standard_normal((3, 3, DQK), dtype=np.float32))
+    return inp, bt, new
+
+
+def test_append_writes_rows_at_the_sequence_ends_only():
+    inp, bt, new = _append_case()
+    kv = oracle.append(new, inp["kv"], bt, inp["seqlens"])
+    flat, old = kv.reshape(-1, DQK), inp["kv"].reshape(-1, DQK)
+    touched = set()
+    for b, n in enumerate(inp["seqlens"]):
+        for t in range(3):
+            pos = int(n) + t
+            row = bt[b, pos // BLK] * BLK + pos % BLK
+            assert np.array_equal(flat[row], new[b, t])
+            touched.add(int(row))
+    rest = np.array([r for r in range(flat.shape[0]) if r not in touched])
+    assert np.array_equal(flat[rest], old[rest])
+
+
+def test_fp8_append_decodes_back_within_e4m3_rounding():
+    inp, bt, new = _append_case("fp8")
+    sc = inp["kv_scale"]
+    kv8 = oracle.append_fp8(new, inp["kv8"], np.float32(1.0 / sc), bt, inp["seqlens"])
+    flat = kv8.reshape(-1, REC)
+    for b, n in enumerate(inp["seqlens"]):
+        for t in range(3):
+            pos = int(n) + t
+            rec = flat[bt[b, pos // BLK] * BLK + pos % BLK]
+            x = W.bf16_bits_to_f32(new[b, t]).astype(np.float64)
+            lat = oracle.e4m3_decode(rec[:DV]) * sc
+            # E4M3 keeps 4 significant bits: relative error <= 2^-4 (normal range), absolute <= 2^-10 sc
+            err = np.abs(lat - x[:DV])
+            assert np.all(err <= np.maximum(np.abs(x[:DV]) * 2.0 ** -4, 2.0 ** -10 * sc) + 1e-12)
+            assert np.array_equal(np.ascontiguousarray(rec[DV:]).view("<u2"), new[b, t, DV:])
