@@ -90,14 +90,16 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
+SPLIT_KERNEL_SOURCES = ("common.cuh", "decode_sm100.cu", "sm100_ptx.cuh")  # the split kernel's device code
+
+
 def kernel_source_hash() -> str:
-    """Hash of the code (not the comments) of the library's CUDA sources."""
+    """Hash of the code (not the comments) of the split kernel's device sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_decode_attention_14_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), encoding="utf-8") as f:
-                h.update((name + "\n" + _code_only(f.read())).encode())
+    for name in SPLIT_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update((name + "\n" + _code_only(f.read())).encode())
     return h.hexdigest()[:16]
 
 

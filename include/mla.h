@@ -186,6 +186,31 @@ int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_bl
                          float *lse, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Appending new tokens to the paged cache, the step that precedes decode. Token t of sequence b's
+ * new tokens goes to position p = seqlens[b] + t of that sequence, i.e. cache row
+ * block_table[b][p / 64] * 64 + p % 64 ("Deep analysis of the DeepSeek Infra open-source releases",
+ * DAY1 FlashMLA, feature (2): 64-token blocks).
+ *   new_kv       bf16[batch, n_new, 576], contiguous, 16-byte aligned: the new tokens' latent vectors
+ *   kv_cache     bf16[num_blocks, 64, 1, 576] (mla_append_kv) or uint8[num_blocks, 64, 1, 640]
+ *                (mla_append_kv_fp8), 16-byte aligned; written in place
+ *   block_table  int32[batch, bt_stride]; the entries for the new positions must already be set
+ *   seqlens      int32[batch]: the lengths BEFORE the append (the caller adds n_new afterwards)
+ *   kv_scale     fp8 only: the cache's latent scale; each latent value x is stored as the E4M3 code
+ *                of x * (1 / kv_scale) (one fp32 multiply), rounded to nearest even and saturated
+ *                to +-448; the rotary dims are stored as bf16
+ * Asynchronous on `stream`; allocates nothing. n_new = 0 is a no-op. A new row whose table entry is
+ * past bt_stride or outside [0, num_blocks) is skipped and reported as MLA_ERR_BOUNDS by
+ * mla_check_status. Returns MLA_ERR_INVALID_ARG for null or misaligned pointers or sizes out of
+ * range (and a non-finite or non-positive kv_scale), MLA_ERR_UNSUPPORTED without an sm_100 device,
+ * MLA_ERR_CUDA if the launch fails, else MLA_OK.
+ */
+int mla_append_kv(const void *new_kv, int n_new, void *kv_cache, int64_t num_blocks, const int32_t *block_table,
+                  int64_t bt_stride, const int32_t *seqlens, int batch, void *stream);
+int mla_append_kv_fp8(const void *new_kv, int n_new, void *kv_cache_fp8, int64_t num_blocks, float kv_scale,
+                      const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens, int batch,
+                      void *stream);
+
+/*
  * End-to-end call on HOST buffers: copies the inputs host->device, runs metadata +
  * decode, copies out/lse device->host, and synchronises `stream` before returning.
  * Host buffers should be pinned for the copies to be asynchronous. `dev` holds the

@@ -40,7 +40,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # exported C symbols, in the order include/mla.h declares them
 EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
            "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_fp8",
-           "mla_decode_split_fp8", "mla_decode_host",
+           "mla_decode_split_fp8", "mla_append_kv", "mla_append_kv_fp8", "mla_decode_host",
            "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_selftest_wait_timeout")
 
 
@@ -85,6 +85,10 @@ def lib():
         for name in ("mla_decode_fp8", "mla_decode_split_fp8"):
             getattr(L, name).argtypes = dec8
             getattr(L, name).restype = I
+        L.mla_append_kv.argtypes = [P, I, P, I64, P, I64, P, I, P]
+        L.mla_append_kv.restype = I
+        L.mla_append_kv_fp8.argtypes = [P, I, P, I64, F, P, I64, P, I, P]
+        L.mla_append_kv_fp8.restype = I
         L.mla_decode_noalloc.argtypes = dec[:16] + [P]
         L.mla_decode_noalloc.restype = I
         L.mla_decode_combine.argtypes = [P, I, I, I, I, P, P, P, SZ, P]
@@ -202,6 +206,51 @@ def _outputs(b, s_q, h_q, meta, dev, out, lse, workspace):
     if workspace.numel() * workspace.element_size() < ws_bytes:
         raise ValueError("workspace too small: need %d bytes" % ws_bytes)
     return out, lse, workspace, ws_bytes
+
+
+def _append_args(new_kv, block_table, seqlens):
+    _need(new_kv, "new_kv", torch.bfloat16, 3)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    b, n_new, d = new_kv.shape
+    if d != D_QK:
+        raise ValueError("new_kv last dim must be %d" % D_QK)
+    if block_table.shape[0] != b or seqlens.shape[0] != b:
+        raise ValueError("batch mismatch between new_kv, block_table and seqlens")
+    return b, n_new  # n_new == 0 is a no-op (an empty tensor may have no storage to point at)
+
+
+def append_kv(new_kv: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+              stream=None) -> None:
+    """Write ``new_kv`` (bf16 ``[b, n_new, 576]``) into the bf16 cache at positions
+    ``seqlens[b] + t`` (``mla_append_kv``); ``seqlens`` are the lengths before the append."""
+    b, n_new = _append_args(new_kv, block_table, seqlens)
+    _need(kv_cache, "kv_cache", torch.bfloat16)
+    if kv_cache.shape[-1] != D_QK or kv_cache.shape[1] != BLOCK:
+        raise ValueError("kv_cache must be [num_blocks, 64, 1, 576]")
+    if n_new == 0:
+        return
+    with torch.cuda.device(new_kv.device):
+        _check("mla_append_kv", lib().mla_append_kv(new_kv.data_ptr(), n_new, kv_cache.data_ptr(), kv_cache.shape[0],
+                                                    block_table.data_ptr(), block_table.shape[1], seqlens.data_ptr(),
+                                                    b, _stream(stream)))
+
+
+def append_kv_fp8(new_kv: torch.Tensor, kv_cache_fp8: torch.Tensor, block_table: torch.Tensor,
+                  seqlens: torch.Tensor, kv_scale: float, stream=None) -> None:
+    """The same into the fp8 cache (``mla_append_kv_fp8``): latent values stored as E4M3 codes of
+    ``x * (1 / kv_scale)``, rotary dims as bf16."""
+    b, n_new = _append_args(new_kv, block_table, seqlens)
+    _need(kv_cache_fp8, "kv_cache_fp8", torch.uint8)
+    if kv_cache_fp8.shape[-1] != FP8_RECORD_BYTES or kv_cache_fp8.shape[1] != BLOCK:
+        raise ValueError("kv_cache_fp8 must be uint8 [num_blocks, 64, 1, %d]" % FP8_RECORD_BYTES)
+    if n_new == 0:
+        return
+    with torch.cuda.device(new_kv.device):
+        _check("mla_append_kv_fp8", lib().mla_append_kv_fp8(new_kv.data_ptr(), n_new, kv_cache_fp8.data_ptr(),
+                                                            kv_cache_fp8.shape[0], float(kv_scale),
+                                                            block_table.data_ptr(), block_table.shape[1],
+                                                            seqlens.data_ptr(), b, _stream(stream)))
 
 
 def decode_fp8(q: torch.Tensor, kv_cache_fp8: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,

@@ -20,6 +20,9 @@ cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, 
                            const float *lse_part, cudaStream_t stream);
 cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
                                 bool fp8, cudaStream_t stream);
+cudaError_t launch_append(const __nv_bfloat16 *new_kv, int n_new, void *kv, int64_t num_blocks,
+                          const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens, int batch,
+                          bool fp8, float inv_scale, cudaStream_t stream);
 
 static std::atomic<int64_t> g_launches{0};
 
@@ -357,6 +360,39 @@ int mla_decode_fp8(const void *q, const void *kv_cache_fp8, int64_t num_blocks, 
     if (rc != MLA_OK) return rc;
     return mla_decode_combine(num_splits, num_parts, batch, s_q, h_q, out, lse, workspace,
                               workspace_bytes, stream);
+}
+
+static int append_common(const void *new_kv, int n_new, void *kv, int64_t num_blocks, const int32_t *block_table,
+                         int64_t bt_stride, const int32_t *seqlens, int batch, bool fp8, float inv_scale,
+                         void *stream) {
+    if (!new_kv || !kv || !block_table || !seqlens) return MLA_ERR_INVALID_ARG;
+    if (batch < 1 || batch > MLA_MAX_BATCH || n_new < 0 || n_new > (1 << 20)) return MLA_ERR_INVALID_ARG;
+    if (num_blocks < 1 || num_blocks > (int64_t)(INT32_MAX / MLA_BLOCK_TOKENS)) return MLA_ERR_INVALID_ARG;
+    if (bt_stride < 1 || bt_stride > (int64_t)INT32_MAX) return MLA_ERR_INVALID_ARG;
+    if (!aligned(new_kv, 16) || !aligned(kv, 16) || !aligned(block_table, 4) || !aligned(seqlens, 4))
+        return MLA_ERR_INVALID_ARG;
+    int rc = check_device();
+    if (rc != MLA_OK) return rc;
+    cudaError_t e = launch_append(static_cast<const __nv_bfloat16 *>(new_kv), n_new, kv, num_blocks, block_table,
+                                  bt_stride, seqlens, batch, fp8, inv_scale, static_cast<cudaStream_t>(stream));
+    g_launches.fetch_add(n_new > 0 ? 1 : 0, std::memory_order_relaxed);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_append_kv(const void *new_kv, int n_new, void *kv_cache, int64_t num_blocks, const int32_t *block_table,
+                  int64_t bt_stride, const int32_t *seqlens, int batch, void *stream) {
+    return append_common(new_kv, n_new, kv_cache, num_blocks, block_table, bt_stride, seqlens, batch, false, 0.f,
+                         stream);
+}
+
+int mla_append_kv_fp8(const void *new_kv, int n_new, void *kv_cache_fp8, int64_t num_blocks, float kv_scale,
+                      const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens, int batch,
+                      void *stream) {
+    if (!std::isfinite(kv_scale) || !(kv_scale > 0.f)) return MLA_ERR_INVALID_ARG;
+    const float inv = 1.f / kv_scale;
+    if (!std::isfinite(inv)) return MLA_ERR_INVALID_ARG;
+    return append_common(new_kv, n_new, kv_cache_fp8, num_blocks, block_table, bt_stride, seqlens, batch, true, inv,
+                         stream);
 }
 
 int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_blocks,

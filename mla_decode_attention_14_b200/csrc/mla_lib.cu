@@ -6,3 +6,4 @@
 #include "decode_sm100.cu"
 #include "noalloc.cu"
 #include "selftest.cu"
+#include "append.cu"

@@ -121,3 +121,13 @@ def test_noalloc_scratch_constant_matches_header():
 def test_selftest_bound_is_checked_on_host(L):
     assert L.mla_selftest_wait_timeout(10, None) == 1  # MLA_ERR_INVALID_ARG: bound below 1e5 cycles
     assert L.mla_selftest_wait_timeout(5_000_000_000, None) == 1
+
+
+def test_append_arguments_checked_on_host(L):
+    # null pointers, batch 0, a negative token count, and (fp8) bad scales never reach a launch
+    assert L.mla_append_kv(None, 1, FAKE, 10, FAKE, 4, FAKE, 2, None) == 1
+    assert L.mla_append_kv(FAKE, 1, FAKE, 10, FAKE, 4, FAKE, 0, None) == 1
+    assert L.mla_append_kv(FAKE, -1, FAKE, 10, FAKE, 4, FAKE, 2, None) == 1
+    assert L.mla_append_kv(FAKE + 8, 1, FAKE, 10, FAKE, 4, FAKE, 2, None) == 1
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert L.mla_append_kv_fp8(FAKE, 1, FAKE, 10, bad, FAKE, 4, FAKE, 2, None) == 1
