@@ -211,6 +211,26 @@ int mla_append_kv_fp8(const void *new_kv, int n_new, void *kv_cache_fp8, int64_t
                       void *stream);
 
 /*
+ * The per-head projections on either side of decode attention, as GEMMs on the tensor cores: for
+ * every head h, Y_h (m x n) = X_h (m x k) W_h (k x n) in bf16 with fp32 accumulation, rounded to
+ * bf16 (nearest even). With the up-projections absorbed into the query and the output ("Deep
+ * analysis of the DeepSeek Infra open-source releases", DAY1 FlashMLA: the kernel works on the
+ * latent vectors; feature (4)), the query side is q_latent = q_nope W_UK (k 128, n 512, written
+ * straight into the first 512 dims of q's rows) and the output side is o = o_latent W_UV
+ * (k 512, n 128).
+ *   x   bf16; row r of X_h starts at x + r * ldx + h * x_head_stride (elements)
+ *   w   bf16[heads, k, n], contiguous (W_h row-major)
+ *   y   bf16; row r of Y_h starts at y + r * ldy + h * y_head_stride; written
+ * k and n are multiples of 64; ldx, x_head_stride, ldy, y_head_stride multiples of 8 (16-byte rows);
+ * the head blocks lie inside a row ((heads - 1) * stride + width <= ld); pointers 16-byte aligned.
+ * Asynchronous on `stream`; allocates nothing. Returns MLA_ERR_INVALID_ARG for arguments outside
+ * these rules, MLA_ERR_UNSUPPORTED without an sm_100 device, MLA_ERR_CUDA if a CUDA call fails, else
+ * MLA_OK; a pipeline wait past its bound is reported as MLA_ERR_TIMEOUT by mla_check_status.
+ */
+int mla_head_gemm(const void *x, int64_t ldx, int64_t x_head_stride, const void *w, void *y, int64_t ldy,
+                  int64_t y_head_stride, int m, int n, int k, int heads, void *stream);
+
+/*
  * End-to-end call on HOST buffers: copies the inputs host->device, runs metadata +
  * decode, copies out/lse device->host, and synchronises `stream` before returning.
  * Host buffers should be pinned for the copies to be asynchronous. `dev` holds the

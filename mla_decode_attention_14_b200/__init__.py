@@ -40,7 +40,8 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # exported C symbols, in the order include/mla.h declares them
 EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
            "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_fp8",
-           "mla_decode_split_fp8", "mla_append_kv", "mla_append_kv_fp8", "mla_decode_host",
+           "mla_decode_split_fp8", "mla_append_kv", "mla_append_kv_fp8", "mla_head_gemm",
+           "mla_decode_host",
            "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_selftest_wait_timeout")
 
 
@@ -89,6 +90,8 @@ def lib():
         L.mla_append_kv.restype = I
         L.mla_append_kv_fp8.argtypes = [P, I, P, I64, F, P, I64, P, I, P]
         L.mla_append_kv_fp8.restype = I
+        L.mla_head_gemm.argtypes = [P, I64, I64, P, P, I64, I64, I, I, I, I, P]
+        L.mla_head_gemm.restype = I
         L.mla_decode_noalloc.argtypes = dec[:16] + [P]
         L.mla_decode_noalloc.restype = I
         L.mla_decode_combine.argtypes = [P, I, I, I, I, P, P, P, SZ, P]
@@ -251,6 +254,45 @@ def append_kv_fp8(new_kv: torch.Tensor, kv_cache_fp8: torch.Tensor, block_table:
                                                             kv_cache_fp8.shape[0], float(kv_scale),
                                                             block_table.data_ptr(), block_table.shape[1],
                                                             seqlens.data_ptr(), b, _stream(stream)))
+
+
+def head_gemm(x: torch.Tensor, ldx: int, x_head_stride: int, w: torch.Tensor, y: torch.Tensor, ldy: int,
+              y_head_stride: int, m: int, n: int, k: int, heads: int, stream=None) -> torch.Tensor:
+    """Per-head GEMM ``Y_h = X_h W_h`` (``mla_head_gemm``); strides in elements, see include/mla.h."""
+    _need(x, "x", torch.bfloat16)
+    _need(w, "w", torch.bfloat16)
+    _need(y, "y", torch.bfloat16)
+    if w.numel() != heads * k * n:
+        raise ValueError("w must hold heads x k x n values")
+    with torch.cuda.device(x.device):
+        _check("mla_head_gemm", lib().mla_head_gemm(x.data_ptr(), ldx, x_head_stride, w.data_ptr(), y.data_ptr(), ldy,
+                                                    y_head_stride, m, n, k, heads, _stream(stream)))
+    return y
+
+
+def absorb_q(q_nope: torch.Tensor, w_uk: torch.Tensor, q: torch.Tensor, stream=None) -> torch.Tensor:
+    """Latent queries ``q[..., :512] = q_nope W_UK`` per head: ``q_nope`` bf16 ``[b, s_q, h, k]``,
+    ``w_uk`` bf16 ``[h, k, 512]``, ``q`` the decode's bf16 ``[b, s_q, h, 576]`` (its rotary dims are
+    left as they are)."""
+    _need(q_nope, "q_nope", torch.bfloat16, 4)
+    _need(q, "q", torch.bfloat16, 4)
+    b, s_q, h, k = q_nope.shape
+    if tuple(q.shape) != (b, s_q, h, D_QK) or tuple(w_uk.shape) != (h, k, D_V):
+        raise ValueError("shapes: q_nope [b, s_q, h, k], w_uk [h, k, 512], q [b, s_q, h, 576]")
+    return head_gemm(q_nope, h * k, k, w_uk, q, h * D_QK, D_QK, b * s_q, D_V, k, h, stream)
+
+
+def absorb_o(o_latent: torch.Tensor, w_uv: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """Per-head output projection ``o = o_latent W_UV``: ``o_latent`` bf16 ``[b, s_q, h, 512]`` (the
+    decode's output), ``w_uv`` bf16 ``[h, 512, d]``; returns bf16 ``[b, s_q, h, d]``."""
+    _need(o_latent, "o_latent", torch.bfloat16, 4)
+    b, s_q, h, k = o_latent.shape
+    if k != D_V or w_uv.dim() != 3 or tuple(w_uv.shape[:2]) != (h, D_V):
+        raise ValueError("shapes: o_latent [b, s_q, h, 512], w_uv [h, 512, d]")
+    d = w_uv.shape[2]
+    if out is None:
+        out = torch.empty((b, s_q, h, d), dtype=torch.bfloat16, device=o_latent.device)
+    return head_gemm(o_latent, h * D_V, D_V, w_uv, out, h * d, d, b * s_q, d, D_V, h, stream)
 
 
 def decode_fp8(q: torch.Tensor, kv_cache_fp8: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,

@@ -20,6 +20,8 @@ cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, 
                            const float *lse_part, cudaStream_t stream);
 cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
                                 bool fp8, cudaStream_t stream);
+cudaError_t launch_head_gemm(const CUtensorMap &map_x, const CUtensorMap &map_w, __nv_bfloat16 *y, int64_t ldy,
+                             int64_t y_head, int64_t x_head, int m, int n, int k, int heads, cudaStream_t stream);
 cudaError_t launch_append(const __nv_bfloat16 *new_kv, int n_new, void *kv, int64_t num_blocks,
                           const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens, int batch,
                           bool fp8, float inv_scale, cudaStream_t stream);
@@ -393,6 +395,38 @@ int mla_append_kv_fp8(const void *new_kv, int n_new, void *kv_cache_fp8, int64_t
     if (!std::isfinite(inv)) return MLA_ERR_INVALID_ARG;
     return append_common(new_kv, n_new, kv_cache_fp8, num_blocks, block_table, bt_stride, seqlens, batch, true, inv,
                          stream);
+}
+
+int mla_head_gemm(const void *x, int64_t ldx, int64_t x_head_stride, const void *w, void *y, int64_t ldy,
+                  int64_t y_head_stride, int m, int n, int k, int heads, void *stream) {
+    if (!x || !w || !y) return MLA_ERR_INVALID_ARG;
+    if (m < 1 || m > (1 << 24) || heads < 1 || heads > 4096) return MLA_ERR_INVALID_ARG;
+    if (k < 64 || k > 65536 || k % 64 != 0 || n < 64 || n > 65536 || n % 64 != 0) return MLA_ERR_INVALID_ARG;
+    if (ldx % 8 || x_head_stride % 8 || ldy % 8 || y_head_stride % 8 || x_head_stride < 0 || y_head_stride < 0)
+        return MLA_ERR_INVALID_ARG;  // rows and head blocks start on 16-byte boundaries
+    const int64_t x_cols = (int64_t)(heads - 1) * x_head_stride + k;
+    if (ldx < x_cols || ldy < (int64_t)(heads - 1) * y_head_stride + n || x_cols > INT32_MAX)
+        return MLA_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16)) return MLA_ERR_INVALID_ARG;
+    int rc = check_device();
+    if (rc != MLA_OK) return rc;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    CUtensorMap map_x, map_w;
+    cuuint64_t dx[2] = {(cuuint64_t)x_cols, (cuuint64_t)m}, sx[1] = {(cuuint64_t)ldx * 2};
+    cuuint64_t dw[2] = {(cuuint64_t)n, (cuuint64_t)heads * k}, sw[1] = {(cuuint64_t)n * 2};
+    cuuint32_t bx[2] = {64, 128}, bw[2] = {64, 64}, estr[2] = {1, 1};
+    if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dx, sx, bx, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), dw, sw, bw, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    cudaError_t e = launch_head_gemm(map_x, map_w, static_cast<__nv_bfloat16 *>(y), ldy, y_head_stride, x_head_stride,
+                                     m, n, k, heads, static_cast<cudaStream_t>(stream));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_blocks,

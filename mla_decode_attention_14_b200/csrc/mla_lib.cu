@@ -7,3 +7,4 @@
 #include "noalloc.cu"
 #include "selftest.cu"
 #include "append.cu"
+#include "head_gemm.cu"

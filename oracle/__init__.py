@@ -200,3 +200,11 @@ def append_fp8(new_kv_bits, kv8, inv_scale: float, block_table, seqlens):
         raise ValueError("oracle_append_fp8: a row lands outside the table or the cache")
     return kv
 
+
+def head_gemm(x, w):
+    """Per-head products in double: ``x`` float ``[m, heads, k]``, ``w`` ``[heads, k, n]`` ->
+    ``[m, heads, n]`` with ``y[r, h] = x[r, h] @ w[h]`` (numpy's matmul as the library step)."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    return np.einsum("mhk,hkn->mhn", x, w)
+

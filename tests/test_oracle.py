@@ -195,3 +195,16 @@ def test_bad_block_id_is_an_error():
     bt[0, 0] = 99
     with pytest.raises(ValueError):
         oracle.decode(inp["q"], inp["kv"], bt, inp["seqlens"], wl.scale, False)
+
+
+def test_head_gemm_matches_brute_force():
+    """The per-head projection oracle against explicit loops (a transposed operand or a wrong head
+    index would show)."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((5, 3, 4))
+    w = rng.standard_normal((3, 4, 6))
+    y = oracle.head_gemm(x, w)
+    for r in range(5):
+        for h in range(3):
+            for n in range(6):
+                assert abs(y[r, h, n] - sum(x[r, h, kk] * w[h, kk, n] for kk in range(4))) < 1e-12
