@@ -259,6 +259,58 @@ def cpu_baseline(wl, inp, target_s=12.0, kv="bf16"):
             "seconds": dt}
 
 
+def neighbour_steps(mla, wl, dev, stream, iters=50):
+    """The steps either side of decode, timed on their own (not part of the step): the per-head
+    projections q_nope W_UK -> q and o_latent W_UV -> o (tcgen05 GEMMs, random weights) and a
+    one-token append into a scratch cache. Each: CUDA-event time per call, algorithmic bytes
+    (weights + activations read once, results written once) and the HBM fraction."""
+    import torch
+    hbm = measured_peaks()[0]
+    b, s_q, h = wl.batch, wl.s_q, wl.h_q
+    g = torch.Generator(device=dev).manual_seed(0)
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=g, device=dev) * scale).to(torch.bfloat16)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    res = {}
+    q_nope, w_uk = rnd(b, s_q, h, 128), rnd(h, 128, 512, scale=128 ** -0.5)
+    q = torch.zeros((b, s_q, h, 576), dtype=torch.bfloat16, device=dev)
+    o_lat, w_uv = rnd(b, s_q, h, 512), rnd(h, 512, 128, scale=512 ** -0.5)
+    rows = b * s_q * h
+    for name, fn, nbytes, flops in (
+            ("absorb_q", lambda: mla.absorb_q(q_nope, w_uk, q), 2 * (h * 128 * 512 + rows * 128 + rows * 512),
+             2 * rows * 128 * 512),
+            ("absorb_o", lambda: mla.absorb_o(o_lat, w_uv), 2 * (h * 512 * 128 + rows * 512 + rows * 128),
+             2 * rows * 512 * 128)):
+        ms = timed(fn)
+        res[name] = {"us": ms * 1e3, "bytes": nbytes, "flops": flops, "GBps": nbytes / (ms * 1e-3) / 1e9,
+                     "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm}
+    new_kv = rnd(b, 1, 576)
+    cache = torch.zeros((b, 64, 1, 576), dtype=torch.bfloat16, device=dev)
+    table = torch.arange(b, dtype=torch.int32, device=dev).reshape(b, 1)
+    lens = torch.zeros((b,), dtype=torch.int32, device=dev)
+    ms = timed(lambda: mla.append_kv(new_kv, cache, table, lens))
+    res["append_kv"] = {"us": ms * 1e3, "bytes": 2 * b * 1152, "GBps": 2 * b * 1152 / (ms * 1e-3) / 1e9}
+    st = mla.check_status()
+    if st != 0:
+        raise SystemExit("device error status %d in the neighbour steps" % st)
+    res["note"] = ("per call, CUDA events, %d calls each; small enough to be launch-bound at this batch: "
+                   "the HBM fraction is of the measured copy peak" % iters)
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -273,6 +325,7 @@ def main():
                     help="replays of the step captured in a CUDA graph, reported under 'graph' "
                          "(default: as many as --steps; 0: skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-neighbours", action="store_true", help="skip timing the projections and the append")
     ap.add_argument("--max-batch", type=int, default=0,
                     help="keep only the first N sequences (for profiler captures of a smaller slice)")
     args = ap.parse_args()
@@ -481,6 +534,8 @@ def main():
         e2e = {"value": bytes_all / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    neighbours = None if args.no_neighbours or fp8 else neighbour_steps(mla, wl, dev, stream)
+
     if rank == 0:
         hbm, tfl_burst, tfl_sust, src = measured_peaks()
         ai = counts["flops"] / counts["bytes"]
@@ -511,6 +566,7 @@ def main():
                                   "steps, outside the timed steps" % (in_bytes / 1e6)),
                            "parallelism": "independent batch per GPU" if world > 1 else "1 GPU"},
                 "roofline": roof, "clocks": clk.summary(), "e2e": e2e, "gpu_launches": launches,
+                "neighbours": neighbours,
                 "graph": None if graph_ms is None else {
                     "ms_per_step": graph_ms, "value": job_throughput(counts["bytes"], world, graph_ms), "unit": "TB/s",
                     "note": "the same step (metadata + split + combine) captured once in a CUDA graph and replayed"}}
