@@ -48,6 +48,14 @@
 //    only touch TMEM lane quarter w & 3). Warpgroup 0 hands registers to the softmax warps.
 //  * Pieces of split sequences leave fp32 partial O and lse in the workspace for the combine
 //    kernel; whole sequences are written straight to bf16 out / fp32 lse.
+//  * The two softmax warps of an SM sub-partition move in lockstep (the per-row barrier) and
+//    share its issue slots, so their instruction count sets the pace: the per-token-pair
+//    arithmetic uses the packed f32x2 instructions and block maxima the three-input max.
+//  * The same kernel, instantiated with F8 = true, reads an FP8 latent cache (640-byte token
+//    records: 512 E4M3 latent bytes, 64 bf16 rotary dims): TMA loads the E4M3 boxes into the
+//    upper half of each stage, four converter warps (warps 4-7) expand them in place to the fp16
+//    layout above, Gemm1's latent MMAs and Gemm2 run in fp16, and P is a single fp16 term set
+//    against the exact block max; the softmax warps are then warps 8-15.
 // Every wait is bounded; a timeout sets the device error word and the CTA exits cleanly.
 #include <cuda_fp16.h>
 
