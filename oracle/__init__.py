@@ -60,6 +60,10 @@ def _load():
         lib.oracle_decode_fp8.restype = ctypes.c_int
         lib.oracle_e4m3_decode.argtypes = [P, ctypes.c_int64, P]
         lib.oracle_e4m3_decode.restype = None
+        lib.oracle_decode_sparse.argtypes = [P, P, ctypes.c_int64, P, ctypes.c_int64, P, P, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, P, P,
+                                             ctypes.c_int]
+        lib.oracle_decode_sparse.restype = ctypes.c_int
         lib.oracle_e4m3_encode.argtypes = [P, ctypes.c_int64, P]
         lib.oracle_e4m3_encode.restype = None
         lib.oracle_append.argtypes = [P, ctypes.c_int, P, ctypes.c_int64, P, ctypes.c_int64, P, ctypes.c_int]
@@ -207,4 +211,26 @@ def head_gemm(x, w):
     x = np.asarray(x, dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
     return np.einsum("mhk,hkn->mhn", x, w)
+
+
+def decode_sparse(q_bits, kv_bits, block_table, seqlens, indices, scale: float, nthreads: int | None = None):
+    """Exact (double) sparse decode: row (b, t, h) attends to the keys at positions
+    ``indices[b, t, :]`` (int32 ``[b, s_q, topk]``; entries outside ``[0, seqlens[b])`` are no key).
+    Returns ``(out float64[b, s_q, h_q, 512], lse float64[b, h_q, s_q])``."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kv = np.ascontiguousarray(kv_bits, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    ix = np.ascontiguousarray(indices, dtype=np.int32)
+    b, s_q, h_q, d = q.shape
+    assert d == D_QK and ix.shape[:2] == (b, s_q)
+    out = np.full((b, s_q, h_q, D_V), np.nan, dtype=np.float64)
+    lse = np.full((b, h_q, s_q), np.nan, dtype=np.float64)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().oracle_decode_sparse(_ptr(q), _ptr(kv), kv.shape[0], _ptr(bt), bt.shape[1], _ptr(sl), _ptr(ix),
+                                      ix.shape[2], b, s_q, h_q, float(scale), _ptr(out), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_decode_sparse failed (rc=%d)" % rc)
+    return out, lse
 

@@ -30,6 +30,12 @@
  * and values are those dequantized vectors; everything after that is the same
  * attention, in double.
  *
+ * Sparse mode (oracle_decode_sparse): query row (b, t, h) attends only to the keys at the
+ * positions listed for query token t of sequence b (shared by its heads); entries outside the
+ * sequence are no key. Pinned in tests/test_oracle_sparse.py (the full list in order is the
+ * dense decode bit for bit; list order and invalid entries change nothing; one key, no key;
+ * a library SDPA over the gathered keys).
+ *
  * Parity pins (see tests/test_oracle*.py): dense non-paged brute force through a
  * library softmax-attention routine, single-token sequences, block-permutation
  * invariance, lse against a library log-sum-exp, q = 0 closed form, NaN-poisoned
@@ -179,6 +185,8 @@ typedef struct {
     double scale;
     double *out, *lse;
     const int32_t *tasks; /* optional list of (b, t, h) triples */
+    const int32_t *indices; /* sparse mode: int32[b, s_q, topk] key positions (NULL: dense) */
+    int topk;
     int64_t ntasks;
     int64_t next;         /* shared work counter */
     pthread_mutex_t lock;
@@ -209,7 +217,11 @@ static int one_row(dec_job *J, int b, int t, int h, double *scores, double *acc)
 
     int64_t n = J->seqlens[b] > 0 ? J->seqlens[b] : 0;
     int64_t V = n;
-    if (J->causal) {
+    const int32_t *list = NULL; /* sparse mode: key i of this row is token list[i] (skipped unless in [0, n)) */
+    if (J->indices) {
+        list = J->indices + ((size_t)b * J->s_q + t) * J->topk;
+        V = J->topk;
+    } else if (J->causal) {
         V = n - J->s_q + t + 1;
         if (V < 0) V = 0;
         if (V > n) V = n;
@@ -224,21 +236,33 @@ static int one_row(dec_job *J, int b, int t, int h, double *scores, double *acc)
 
     double m = -INFINITY, key[OR_D_QK];
     for (int64_t j = 0; j < V; ++j) {
-        int32_t phys = J->block_table[(size_t)b * J->bt_stride + j / OR_BLK];
+        const int64_t pos = list ? (int64_t)list[j] : j;
+        if (pos < 0 || pos >= n) { /* sparse mode: an entry outside the sequence is no key */
+            scores[j] = -INFINITY;
+            continue;
+        }
+        int32_t phys = J->block_table[(size_t)b * J->bt_stride + pos / OR_BLK];
         if (phys < 0 || phys >= J->num_blocks) return -1;
-        load_key(J, (int64_t)phys * OR_BLK + j % OR_BLK, key);
+        load_key(J, (int64_t)phys * OR_BLK + pos % OR_BLK, key);
         double dot = 0.0;
         for (int d = 0; d < OR_D_QK; ++d) dot += qd[d] * key[d];
         scores[j] = J->scale * dot;
         if (scores[j] > m) m = scores[j];
+    }
+    if (m == -INFINITY) { /* no valid key */
+        for (int d = 0; d < OR_D_V; ++d) o[d] = 0.0;
+        *lse = -INFINITY;
+        return 0;
     }
     double sum = 0.0;
     for (int64_t j = 0; j < V; ++j) sum += exp(scores[j] - m);
     double L = m + log(sum);
     for (int d = 0; d < OR_D_V; ++d) acc[d] = 0.0;
     for (int64_t j = 0; j < V; ++j) {
-        int32_t phys = J->block_table[(size_t)b * J->bt_stride + j / OR_BLK];
-        load_key(J, (int64_t)phys * OR_BLK + j % OR_BLK, key); /* the value is its first 512 dims */
+        if (scores[j] == -INFINITY) continue;
+        const int64_t pos = list ? (int64_t)list[j] : j;
+        int32_t phys = J->block_table[(size_t)b * J->bt_stride + pos / OR_BLK];
+        load_key(J, (int64_t)phys * OR_BLK + pos % OR_BLK, key); /* the value is its first 512 dims */
         double p = exp(scores[j] - L);
         for (int d = 0; d < OR_D_V; ++d) acc[d] += p * key[d];
     }
@@ -249,7 +273,7 @@ static int one_row(dec_job *J, int b, int t, int h, double *scores, double *acc)
 
 static void *dec_worker(void *arg) {
     dec_job *J = (dec_job *)arg;
-    int64_t maxlen = 0;
+    int64_t maxlen = J->indices ? J->topk : 0;
     for (int b = 0; b < J->batch; ++b)
         if (J->seqlens[b] > maxlen) maxlen = J->seqlens[b];
     double *scores = (double *)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
@@ -451,5 +475,42 @@ int oracle_append_fp8(const uint16_t *new_kv, int n_new, uint8_t *kv8, float inv
                       const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens, int batch) {
     if (!kv8) return -1;
     return append_rows(new_kv, n_new, NULL, kv8, inv_scale, num_blocks, block_table, bt_stride, seqlens, batch);
+}
+
+/*
+ * Sparse mode: query row (b, t, h) attends only to the keys at the positions
+ * indices[b][t][0 .. topk) of sequence b (shared by every head of that query token). An entry
+ * outside [0, seqlens[b]) is no key; an entry listed twice counts twice; a row with no valid
+ * entry gives out = 0, lse = -inf. No causal mask (the list decides). bf16 cache; other
+ * arguments and return codes as oracle_decode.
+ */
+int oracle_decode_sparse(const uint16_t *q, const uint16_t *kv_cache, int64_t num_blocks,
+                         const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
+                         const int32_t *indices, int topk, int batch, int s_q, int h_q, double scale,
+                         double *out, double *lse, int nthreads) {
+    if (!q || !kv_cache || !block_table || !seqlens || !indices || !out || !lse) return -1;
+    if (batch < 0 || s_q < 1 || h_q < 1 || nthreads < 1 || num_blocks < 0 || topk < 0) return -1;
+    for (int b = 0; b < batch; ++b) {
+        int64_t n = seqlens[b] > 0 ? seqlens[b] : 0;
+        if ((n + OR_BLK - 1) / OR_BLK > bt_stride) return -1;
+    }
+    dec_job J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.kv = kv_cache; J.num_blocks = num_blocks; J.block_table = block_table;
+    J.bt_stride = bt_stride; J.seqlens = seqlens; J.batch = batch; J.s_q = s_q; J.h_q = h_q;
+    J.causal = 0; J.scale = scale; J.out = out; J.lse = lse; J.indices = indices; J.topk = topk;
+    pthread_mutex_init(&J.lock, NULL);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) return -2;
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, dec_worker, &J) != 0) break;
+        ++started;
+    }
+    if (started == 0) dec_worker(&J);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return J.error;
 }
 
