@@ -131,3 +131,16 @@ def test_append_arguments_checked_on_host(L):
     assert L.mla_append_kv(FAKE + 8, 1, FAKE, 10, FAKE, 4, FAKE, 2, None) == 1
     for bad in (0.0, -1.0, float("nan"), float("inf")):
         assert L.mla_append_kv_fp8(FAKE, 1, FAKE, 10, bad, FAKE, 4, FAKE, 2, None) == 1
+
+
+def test_head_gemm_arguments_checked_on_host(L):
+    ok = dict(x=FAKE, ldx=2048, xh=128, w=FAKE, y=FAKE, ldy=8192, yh=512, m=4, n=512, k=128, heads=16)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return L.mla_head_gemm(a["x"], a["ldx"], a["xh"], a["w"], a["y"], a["ldy"], a["yh"], a["m"], a["n"], a["k"],
+                               a["heads"], None)
+    for bad in (dict(x=None), dict(w=None), dict(y=None), dict(m=0), dict(heads=0), dict(k=96), dict(n=100),
+                dict(ldx=2044), dict(xh=100), dict(ldx=1024), dict(ldy=4096), dict(x=FAKE + 8)):
+        assert call(**bad) == 1, bad  # MLA_ERR_INVALID_ARG
