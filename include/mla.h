@@ -31,14 +31,19 @@
  *      accumulators (same section, feature (4)), an fp32 online softmax; pieces of
  *      split sequences leave fp32 partial outputs + lse in the workspace, and a
  *      combine kernel merges them by log-sum-exp.
+ * Around it: mla_decode_fp8 reads an FP8 (E4M3) latent cache instead; mla_append_kv /
+ * mla_append_kv_fp8 write new tokens into the cache; mla_head_gemm computes the per-head
+ * projections on either side (the absorbed q_nope W_UK and o_latent W_UV); mla_decode_host
+ * and mla_decode_noalloc are conveniences over mla_decode.
  *
  * Conventions for every call:
  *   - Pointers are DEVICE pointers unless the name says host. All device buffers are
  *     owned by the caller; the library allocates no device memory. It keeps only a
- *     small host-side cache of TMA descriptors keyed by (kv_cache, num_blocks).
+ *     small host-side cache of TMA descriptors keyed by (kv_cache, num_blocks, format).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *     asynchronous unless stated; nothing is synchronised implicitly.
- *   - Inputs are never written. Arguments are validated on the host BEFORE any launch;
+ *   - Inputs are never written (the cache appends write the cache, their output). Arguments
+ *     are validated on the host BEFORE any launch;
  *     an invalid call returns a non-zero mla_status and launches nothing.
  *   - Kernels never trap. A block-table entry outside [0, num_blocks) or a pipeline
  *     wait that exceeds its iteration bound sets a per-device error word; the affected
