@@ -485,48 +485,11 @@ def main():
 
     # end to end through the host entry point: pinned host inputs in, host outputs out
     e2e = None
-    if args.e2e_steps > 0 and fp8:
-        # the fp8 path has no host entry point: the same work through the Python API, each step
-        # copying the inputs from pinned host memory and the results back, then synchronising
-        qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
-        kvh = torch.from_numpy(inp["kv8"]).pin_memory()
-        bth = torch.from_numpy(inp["block_table"]).pin_memory()
-        slh = torch.from_numpy(inp["seqlens"]).pin_memory()
-        oh = torch.empty(tuple(out.shape), dtype=torch.bfloat16).pin_memory()
-        lh = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
-        qd, kvd, btd, sld = torch.empty_like(q), torch.empty_like(kv), torch.empty_like(bt), torch.empty_like(sl)
-
-        def host_step():
-            for d, h in ((qd, qh), (kvd, kvh), (btd, bth), (sld, slh)):
-                d.copy_(h, non_blocking=True)
-            meta = mla.get_metadata(sld, wl.h_q, wl.s_q, num_parts=num_parts, fixed_cost=fixed_cost)
-            decode(qd, kvd, btd, sld, meta, out, lse, ws, "both")
-            oh.copy_(out, non_blocking=True)
-            lh.copy_(lse, non_blocking=True)
-            stream.synchronize()
-
-        for _ in range(2):
-            host_step()
-        if dist is not None:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            host_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dev)[0]
-        h2d = sum(x.numel() * x.element_size() for x in (qh, kvh, bth, slh))
-        d2h = oh.numel() * 2 + lh.numel() * 4
-        e2e = {"value": bytes_all / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": "Python API (decode_fp8) with pinned-host copies in and out, synchronised every step"}
-    elif args.e2e_steps > 0:
+    if args.e2e_steps > 0:
         hd = mla.HostDecoder(wl.batch, wl.s_q, wl.h_q, kv.shape[0], bt.shape[1], device=dev,
-                             num_parts=num_parts, fixed_cost=fixed_cost)
+                             num_parts=num_parts, fixed_cost=fixed_cost, kv_scale=inp["kv_scale"] if fp8 else None)
         qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
-        kvh = torch.from_numpy(inp["kv"]).view(torch.bfloat16).pin_memory()
+        kvh = (torch.from_numpy(inp["kv8"]) if fp8 else torch.from_numpy(inp["kv"]).view(torch.bfloat16)).pin_memory()
         bth = torch.from_numpy(inp["block_table"]).pin_memory()
         slh = torch.from_numpy(inp["seqlens"]).pin_memory()
         oh = torch.empty(tuple(out.shape), dtype=torch.bfloat16).pin_memory()

@@ -263,6 +263,12 @@ int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_b
                     const int32_t *seqlens_host, int batch, int s_q, int h_q, float scale,
                     int causal, void *out_host, float *lse_host,
                     const mla_device_buffers *dev, void *stream);
+/* The same over the fp8 cache (mla_decode_fp8): kv_cache_fp8_host is uint8[num_blocks, 64, 1,
+ * MLA_FP8_RECORD_BYTES] and dev->kv_cache a device buffer of that size. */
+int mla_decode_host_fp8(const void *q_host, const void *kv_cache_fp8_host, int64_t num_blocks, float kv_scale,
+                        const int32_t *block_table_host, int64_t bt_stride, const int32_t *seqlens_host,
+                        int batch, int s_q, int h_q, float scale, int causal, void *out_host, float *lse_host,
+                        const mla_device_buffers *dev, void *stream);
 
 /*
  * Decode for callers that cannot allocate device memory (no counterpart on the pages: this

@@ -41,7 +41,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
            "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_fp8",
            "mla_decode_split_fp8", "mla_append_kv", "mla_append_kv_fp8", "mla_head_gemm",
-           "mla_decode_host",
+           "mla_decode_host", "mla_decode_host_fp8",
            "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_selftest_wait_timeout")
 
 
@@ -99,6 +99,9 @@ def lib():
         L.mla_decode_host.argtypes = [P, P, I64, P, I64, P, I, I, I, F, I, P, P,
                                       ctypes.POINTER(_DeviceBuffers), P]
         L.mla_decode_host.restype = I
+        L.mla_decode_host_fp8.argtypes = [P, P, I64, F, P, I64, P, I, I, I, F, I, P, P,
+                                          ctypes.POINTER(_DeviceBuffers), P]
+        L.mla_decode_host_fp8.restype = I
         L.mla_check_status.argtypes = [P]
         L.mla_check_status.restype = I
         L.mla_launch_count.argtypes = []
@@ -401,14 +404,17 @@ class HostDecoder:
     Device buffers are allocated once (by torch) for the largest shapes given.
     """
 
-    def __init__(self, batch, s_q, h_q, num_blocks, bt_stride, device="cuda", num_parts=None, fixed_cost=None):
+    def __init__(self, batch, s_q, h_q, num_blocks, bt_stride, device="cuda", num_parts=None, fixed_cost=None,
+                 kv_scale=None):
         dev = torch.device(device)
+        self.kv_scale = kv_scale  # not None: the fp8 cache (mla_decode_host_fp8)
         self.device = dev
         self.num_parts = num_parts or default_num_parts(h_q, s_q, dev)
         self.fixed_cost = default_fixed_cost(h_q, s_q) if fixed_cost is None else fixed_cost
         e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)  # noqa: E731
         self.q = e((batch, s_q, h_q, D_QK), torch.bfloat16)
-        self.kv = e((num_blocks, BLOCK, 1, D_QK), torch.bfloat16)
+        self.kv = (e((num_blocks, BLOCK, 1, FP8_RECORD_BYTES), torch.uint8) if kv_scale is not None
+                   else e((num_blocks, BLOCK, 1, D_QK), torch.bfloat16))
         self.bt = e((batch, bt_stride), torch.int32)
         self.sl = e((batch,), torch.int32)
         self.tm = e((self.num_parts, META_INTS), torch.int32)
@@ -429,10 +435,16 @@ class HostDecoder:
                 raise ValueError("%s must be a contiguous host tensor" % n)
         b, s_q, h_q, _ = q.shape
         with torch.cuda.device(self.device):
-            _check("mla_decode_host", lib().mla_decode_host(
-                q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(), block_table.shape[1],
-                seqlens.data_ptr(), b, s_q, h_q, float(scale), int(bool(causal)), out.data_ptr(), lse.data_ptr(),
-                ctypes.byref(self.buf), _stream(stream)))
+            if self.kv_scale is not None:
+                _check("mla_decode_host_fp8", lib().mla_decode_host_fp8(
+                    q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], float(self.kv_scale), block_table.data_ptr(),
+                    block_table.shape[1], seqlens.data_ptr(), b, s_q, h_q, float(scale), int(bool(causal)),
+                    out.data_ptr(), lse.data_ptr(), ctypes.byref(self.buf), _stream(stream)))
+            else:
+                _check("mla_decode_host", lib().mla_decode_host(
+                    q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(),
+                    block_table.shape[1], seqlens.data_ptr(), b, s_q, h_q, float(scale), int(bool(causal)),
+                    out.data_ptr(), lse.data_ptr(), ctypes.byref(self.buf), _stream(stream)))
         return out, lse
 
 

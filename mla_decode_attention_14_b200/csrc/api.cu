@@ -429,18 +429,18 @@ int mla_head_gemm(const void *x, int64_t ldx, int64_t x_head_stride, const void 
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_blocks,
-                    const int32_t *block_table_host, int64_t bt_stride,
-                    const int32_t *seqlens_host, int batch, int s_q, int h_q, float scale,
-                    int causal, void *out_host, float *lse_host,
-                    const mla_device_buffers *dev, void *stream) {
+static int decode_host_common(const void *q_host, const void *kv_cache_host, int64_t num_blocks, bool fp8,
+                              float kv_scale, const int32_t *block_table_host, int64_t bt_stride,
+                              const int32_t *seqlens_host, int batch, int s_q, int h_q, float scale, int causal,
+                              void *out_host, float *lse_host, const mla_device_buffers *dev, void *stream) {
     if (!q_host || !kv_cache_host || !block_table_host || !seqlens_host || !out_host || !lse_host || !dev)
         return MLA_ERR_INVALID_ARG;
     if (!shape_ok(batch, s_q, h_q) || num_blocks < 1 || bt_stride < 1) return MLA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int rows = s_q * h_q;
     const size_t q_bytes = (size_t)batch * rows * MLA_D_QK * 2;
-    const size_t kv_bytes = (size_t)num_blocks * MLA_BLOCK_TOKENS * MLA_D_QK * 2;
+    const size_t kv_bytes =
+        (size_t)num_blocks * MLA_BLOCK_TOKENS * (fp8 ? (size_t)MLA_FP8_RECORD_BYTES : (size_t)MLA_D_QK * 2);
     const size_t bt_bytes = (size_t)batch * bt_stride * sizeof(int32_t);
     const size_t sl_bytes = (size_t)batch * sizeof(int32_t);
     const size_t out_bytes = (size_t)batch * rows * MLA_D_V * 2;
@@ -458,14 +458,36 @@ int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_b
     rc = mla_get_metadata(dev->seqlens, batch, h_q, s_q, dev->num_parts, dev->fixed_cost, dev->tile_meta,
                           dev->num_splits, stream);
     if (rc != MLA_OK) return rc;
-    rc = mla_decode(dev->q, dev->kv_cache, num_blocks, dev->block_table, bt_stride, dev->seqlens,
-                    dev->tile_meta, dev->num_splits, dev->num_parts, batch, s_q, h_q, scale, causal,
-                    dev->out, dev->lse, dev->workspace, dev->workspace_bytes, stream);
+    if (fp8)
+        rc = mla_decode_fp8(dev->q, dev->kv_cache, num_blocks, kv_scale, dev->block_table, bt_stride, dev->seqlens,
+                            dev->tile_meta, dev->num_splits, dev->num_parts, batch, s_q, h_q, scale, causal,
+                            dev->out, dev->lse, dev->workspace, dev->workspace_bytes, stream);
+    else
+        rc = mla_decode(dev->q, dev->kv_cache, num_blocks, dev->block_table, bt_stride, dev->seqlens,
+                        dev->tile_meta, dev->num_splits, dev->num_parts, batch, s_q, h_q, scale, causal,
+                        dev->out, dev->lse, dev->workspace, dev->workspace_bytes, stream);
     if (rc != MLA_OK) return rc;
     if (cudaMemcpyAsync(out_host, dev->out, out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaMemcpyAsync(lse_host, dev->lse, lse_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return MLA_ERR_CUDA;
     return cudaStreamSynchronize(st) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_blocks,
+                    const int32_t *block_table_host, int64_t bt_stride,
+                    const int32_t *seqlens_host, int batch, int s_q, int h_q, float scale,
+                    int causal, void *out_host, float *lse_host,
+                    const mla_device_buffers *dev, void *stream) {
+    return decode_host_common(q_host, kv_cache_host, num_blocks, false, 0.f, block_table_host, bt_stride,
+                              seqlens_host, batch, s_q, h_q, scale, causal, out_host, lse_host, dev, stream);
+}
+
+int mla_decode_host_fp8(const void *q_host, const void *kv_cache_fp8_host, int64_t num_blocks, float kv_scale,
+                        const int32_t *block_table_host, int64_t bt_stride, const int32_t *seqlens_host,
+                        int batch, int s_q, int h_q, float scale, int causal, void *out_host, float *lse_host,
+                        const mla_device_buffers *dev, void *stream) {
+    return decode_host_common(q_host, kv_cache_fp8_host, num_blocks, true, kv_scale, block_table_host, bt_stride,
+                              seqlens_host, batch, s_q, h_q, scale, causal, out_host, lse_host, dev, stream);
 }
 
 int mla_check_status(void *stream) {

@@ -209,3 +209,19 @@ def test_deterministic_and_graph_capturable():
     assert mla.check_status() == 0
     assert torch.equal(og, o1) and torch.equal(lg, l1)
     del graph
+
+
+def test_host_entry_point_matches_device_path():
+    """mla_decode_host_fp8 (host buffers in and out) gives the device path's bits."""
+    wl = W.custom(3, 64, 2, [300, 1, 129], causal=True)
+    inp = W.make_inputs_fp8(wl, seed=9, kv_scale=0.0123)
+    out_d, lse_d, _ = run_fp8(inp)
+    dec = mla.HostDecoder(3, 2, 64, inp["kv8"].shape[0], inp["block_table"].shape[1], kv_scale=inp["kv_scale"])
+    qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
+    kvh = torch.from_numpy(inp["kv8"]).pin_memory()
+    bth = torch.from_numpy(inp["block_table"]).pin_memory()
+    slh = torch.from_numpy(inp["seqlens"]).pin_memory()
+    oh = torch.empty((3, 2, 64, 512), dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty((3, 64, 2), dtype=torch.float32).pin_memory()
+    dec(qh, kvh, bth, slh, inp["scale"], True, oh, lh)
+    assert torch.equal(oh, out_d.cpu()) and torch.equal(lh, lse_d.cpu())
