@@ -152,6 +152,7 @@ cudaError_t launch_head_gemm(const CUtensorMap &map_x, const CUtensorMap &map_w,
     cudaError_t e = cudaFuncSetAttribute(hg::head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)((m + hg::kM - 1) / hg::kM) * heads * ((n + hg::kMaxN - 1) / hg::kMaxN);
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
     hg::head_gemm_kernel<<<(unsigned)grid, 128, smem, stream>>>(map_x, map_w, p);
     return cudaGetLastError();
 }
