@@ -306,6 +306,11 @@ int mla_check_status(void *stream);
  * counter; used to report how many of the library's kernels a benchmark ran). */
 int64_t mla_launch_count(void);
 
+/* Name and description of the last CUDA error that a call of this library saw (a failed
+ * launch, or an earlier asynchronous fault reported by mla_check_status), for the message that
+ * goes with MLA_ERR_CUDA; "no error" if there was none. Host only; the string is static. */
+const char *mla_last_cuda_error(void);
+
 /*
  * Test of the failure path of the kernels' bounded waits (the pages have no counterpart; it
  * exists so that the timeout path can be exercised without a fault). Launches, on `stream`,

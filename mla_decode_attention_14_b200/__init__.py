@@ -42,13 +42,16 @@ EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost
            "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_fp8",
            "mla_decode_split_fp8", "mla_append_kv", "mla_append_kv_fp8", "mla_head_gemm",
            "mla_decode_host", "mla_decode_host_fp8",
-           "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_selftest_wait_timeout")
+           "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_last_cuda_error",
+           "mla_selftest_wait_timeout")
 
 
 class MLAError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
         msg = lib().mla_status_string(status).decode() if _lib is not None else STATUS_NAMES.get(status, "?")
+        if status == 4 and _lib is not None:  # MLA_ERR_CUDA: say which CUDA error it was
+            msg += " [%s]" % lib().mla_last_cuda_error().decode()
         super().__init__("%s failed: %s (status %d)" % (fn, msg, status))
 
 
@@ -106,6 +109,8 @@ def lib():
         L.mla_check_status.restype = I
         L.mla_launch_count.argtypes = []
         L.mla_launch_count.restype = I64
+        L.mla_last_cuda_error.argtypes = []
+        L.mla_last_cuda_error.restype = ctypes.c_char_p
         L.mla_selftest_wait_timeout.argtypes = [I64, P]
         L.mla_selftest_wait_timeout.restype = I
         _lib = L

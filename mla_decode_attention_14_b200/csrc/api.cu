@@ -27,6 +27,14 @@ cudaError_t launch_append(const __nv_bfloat16 *new_kv, int n_new, void *kv, int6
                           bool fp8, float inv_scale, cudaStream_t stream);
 
 static std::atomic<int64_t> g_launches{0};
+static std::atomic<int> g_last_cuda_error{0};  // cudaError_t of the last failing CUDA call
+
+// MLA_OK for cudaSuccess; otherwise remembers the error (see mla_last_cuda_error) -> MLA_ERR_CUDA.
+static int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return 0;
+    g_last_cuda_error.store((int)e, std::memory_order_relaxed);
+    return MLA_ERR_CUDA;
+}
 
 namespace {
 
@@ -52,12 +60,11 @@ int check_device() {
     return st == 1 ? MLA_OK : MLA_ERR_UNSUPPORTED;
 }
 
-// ---- TMA descriptors of the paged cache, viewed as a 2-D bf16 tensor [num_blocks * 64, 576]:
-// "latent" boxes are 64 tokens x 64 dims with the 128-byte swizzle, "rope" boxes are
-// 64 tokens x 32 dims with the 64-byte swizzle (the layouts the MMA descriptors expect).
-// fp8 cache ([num_blocks * 64] records of 640 bytes): "latent" boxes are 64 tokens x 128 bytes
-// (E4M3) with the 128-byte swizzle over a uint8 view, "rope" boxes 64 tokens x 32 bf16 with the
-// 64-byte swizzle over a [rows, 320] bf16 view of the same records.
+// ---- TMA descriptors of the paged cache for the exchange kernel. "latent": the cache viewed as
+// [boxes][rows][box] -- bf16: [9][num_blocks * 64][64 dims], fp8: [5][num_blocks * 64][128 bytes]
+// (E4M3, uint8 view) -- so that ONE operation brings a CTA's 4 bf16 (2 E4M3) latent boxes of
+// 64 tokens x 128 bytes with the 128-byte swizzle; "rope": 64 tokens x 32 bf16 dims with the
+// 64-byte swizzle over a 2-D bf16 view [rows, 288] (bf16) or [rows, 320] (fp8 records).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -107,14 +114,14 @@ int cache_maps(const void *kv, int64_t num_blocks, int fp8, CUtensorMap *lat, CU
     e.fp8 = fp8;
     const cuuint64_t rows = (cuuint64_t)num_blocks * MLA_BLOCK_TOKENS;
     const cuuint64_t rec = fp8 ? (cuuint64_t)MLA_FP8_RECORD_BYTES : (cuuint64_t)MLA_D_QK * 2;
-    cuuint64_t dims[2] = {rec / 2, rows};                    // bf16 view
-    cuuint64_t dims8[2] = {rec, rows};                       // uint8 view (fp8 latent)
+    cuuint64_t dims[2] = {rec / 2, rows};  // bf16 view (rotary boxes)
     cuuint64_t strides[1] = {rec};
-    cuuint32_t box_lat[2] = {64, 64}, box_lat8[2] = {128, 64}, box_rope[2] = {32, 64}, estr[2] = {1, 1};
-    if (enc(&e.lat, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv),
-            fp8 ? dims8 : dims, strides, fp8 ? box_lat8 : box_lat, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    cuuint64_t dims3[3] = {fp8 ? 128u : 64u, rows, fp8 ? 4u : 9u}, strides3[2] = {rec, 128};
+    cuuint32_t box3[3] = {fp8 ? 128u : 64u, 64, fp8 ? 2u : 4u}, estr3[3] = {1, 1, 1};
+    cuuint32_t box_rope[2] = {32, 64}, estr[2] = {1, 1};
+    if (enc(&e.lat, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(kv),
+            dims3, strides3, box3, estr3, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return MLA_ERR_CUDA;
     if (enc(&e.rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv), dims, strides, box_rope, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -256,7 +263,7 @@ int mla_get_metadata(const int32_t *seqlens, int batch, int h_q, int s_q, int nu
     cudaError_t e = launch_metadata(seqlens, batch, num_parts, fixed_cost, tile_meta, num_splits,
                                     static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return cuda_status(e);
 }
 
 int mla_decode_split(const void *q, const void *kv_cache, int64_t num_blocks,
@@ -278,7 +285,7 @@ int mla_decode_split(const void *q, const void *kv_cache, int64_t num_blocks,
     if (rc != MLA_OK) return rc;
     cudaError_t e = launch_decode_sm100(p, map_lat, map_rope, false, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return cuda_status(e);
 }
 
 int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_blocks, float kv_scale,
@@ -315,7 +322,7 @@ int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_bl
     if (rc != MLA_OK) return rc;
     cudaError_t e = launch_decode_sm100(p, map_lat, map_rope, true, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return cuda_status(e);
 }
 
 int mla_decode_combine(const int32_t *num_splits, int num_parts, int batch, int s_q, int h_q,
@@ -335,7 +342,7 @@ int mla_decode_combine(const int32_t *num_splits, int num_parts, int batch, int 
     cudaError_t e = launch_combine(num_splits, batch, num_parts, s_q, h_q, static_cast<__nv_bfloat16 *>(out), lse,
                                    o_part, lse_part, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return cuda_status(e);
 }
 
 int mla_decode(const void *q, const void *kv_cache, int64_t num_blocks,
@@ -378,7 +385,7 @@ static int append_common(const void *new_kv, int n_new, void *kv, int64_t num_bl
     cudaError_t e = launch_append(static_cast<const __nv_bfloat16 *>(new_kv), n_new, kv, num_blocks, block_table,
                                   bt_stride, seqlens, batch, fp8, inv_scale, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(n_new > 0 ? 1 : 0, std::memory_order_relaxed);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return cuda_status(e);
 }
 
 int mla_append_kv(const void *new_kv, int n_new, void *kv_cache, int64_t num_blocks, const int32_t *block_table,
@@ -426,7 +433,7 @@ int mla_head_gemm(const void *x, int64_t ldx, int64_t x_head_stride, const void 
     cudaError_t e = launch_head_gemm(map_x, map_w, static_cast<__nv_bfloat16 *>(y), ldy, y_head_stride, x_head_stride,
                                      m, n, k, heads, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return cuda_status(e);
 }
 
 static int decode_host_common(const void *q_host, const void *kv_cache_host, int64_t num_blocks, bool fp8,
@@ -450,11 +457,12 @@ static int decode_host_common(const void *q_host, const void *kv_cache_host, int
         return MLA_ERR_INVALID_ARG;
     int rc = check_device();
     if (rc != MLA_OK) return rc;
-    if (cudaMemcpyAsync(dev->q, q_host, q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dev->kv_cache, kv_cache_host, kv_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dev->block_table, block_table_host, bt_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dev->seqlens, seqlens_host, sl_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-        return MLA_ERR_CUDA;
+    if ((rc = cuda_status(cudaMemcpyAsync(dev->q, q_host, q_bytes, cudaMemcpyHostToDevice, st))) != MLA_OK ||
+        (rc = cuda_status(cudaMemcpyAsync(dev->kv_cache, kv_cache_host, kv_bytes, cudaMemcpyHostToDevice, st))) != MLA_OK ||
+        (rc = cuda_status(cudaMemcpyAsync(dev->block_table, block_table_host, bt_bytes, cudaMemcpyHostToDevice, st))) !=
+            MLA_OK ||
+        (rc = cuda_status(cudaMemcpyAsync(dev->seqlens, seqlens_host, sl_bytes, cudaMemcpyHostToDevice, st))) != MLA_OK)
+        return rc;
     rc = mla_get_metadata(dev->seqlens, batch, h_q, s_q, dev->num_parts, dev->fixed_cost, dev->tile_meta,
                           dev->num_splits, stream);
     if (rc != MLA_OK) return rc;
@@ -467,10 +475,10 @@ static int decode_host_common(const void *q_host, const void *kv_cache_host, int
                         dev->tile_meta, dev->num_splits, dev->num_parts, batch, s_q, h_q, scale, causal,
                         dev->out, dev->lse, dev->workspace, dev->workspace_bytes, stream);
     if (rc != MLA_OK) return rc;
-    if (cudaMemcpyAsync(out_host, dev->out, out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaMemcpyAsync(lse_host, dev->lse, lse_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return MLA_ERR_CUDA;
-    return cudaStreamSynchronize(st) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    if ((rc = cuda_status(cudaMemcpyAsync(out_host, dev->out, out_bytes, cudaMemcpyDeviceToHost, st))) != MLA_OK ||
+        (rc = cuda_status(cudaMemcpyAsync(lse_host, dev->lse, lse_bytes, cudaMemcpyDeviceToHost, st))) != MLA_OK)
+        return rc;
+    return cuda_status(cudaStreamSynchronize(st));
 }
 
 int mla_decode_host(const void *q_host, const void *kv_cache_host, int64_t num_blocks,
@@ -491,11 +499,12 @@ int mla_decode_host_fp8(const void *q_host, const void *kv_cache_fp8_host, int64
 }
 
 int mla_check_status(void *stream) {
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    int rc = cuda_status(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    if (rc == MLA_OK) rc = cuda_status(cudaGetLastError());
+    if (rc != MLA_OK) return rc;
     unsigned int word = 0, zero = 0;
-    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof word) != cudaSuccess) return MLA_ERR_CUDA;
-    if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero) != cudaSuccess) return MLA_ERR_CUDA;
+    if ((rc = cuda_status(cudaMemcpyFromSymbol(&word, g_error_word, sizeof word))) != MLA_OK) return rc;
+    if (word != 0 && (rc = cuda_status(cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero))) != MLA_OK) return rc;
     if (word & kErrBounds) return MLA_ERR_BOUNDS;
     if (word & kErrTimeout) return MLA_ERR_TIMEOUT;
     if (word & kErrRange) return MLA_ERR_RANGE;
@@ -503,5 +512,10 @@ int mla_check_status(void *stream) {
 }
 
 int64_t mla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *mla_last_cuda_error(void) {
+    const int e = g_last_cuda_error.load(std::memory_order_relaxed);
+    return e == 0 ? "no error" : cudaGetErrorString((cudaError_t)e);
+}
 
 }  // extern "C"

@@ -55,6 +55,7 @@ __device__ __forceinline__ int visible_keys(int n, int s_q, int t, int causal) {
     return v < 0 ? 0 : (v > n ? n : v);
 }
 
-__device__ __forceinline__ int num_blocks_of(int n) { return n > 0 ? (n + kBlk - 1) / kBlk : 0; }
+// ceil(n / 64) without forming n + 63 (which overflows for n near INT32_MAX)
+__device__ __forceinline__ int num_blocks_of(int n) { return n > 0 ? (n - 1) / kBlk + 1 : 0; }
 
 }  // namespace mla

@@ -60,6 +60,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "schedule.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mla {
@@ -124,43 +125,6 @@ struct __align__(1024) Smem {
 
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory (with 1 KB for alignment) must fit 227 KB");
 
-struct Piece {
-    int seq, lo, hi, n, nsplit, slot;
-};
-
-// Walks the non-empty pieces of one part (all roles walk the same list independently).
-struct Cursor {
-    int seq, begin_seq, begin_blk, end_seq, end_blk, first_piece;
-    __device__ void init(const int32_t *meta, int batch) {
-        begin_seq = meta[0];
-        begin_blk = meta[1];
-        end_seq = meta[2];
-        end_blk = meta[3];
-        first_piece = meta[4];
-        if (end_seq >= begin_seq && (begin_seq < 0 || end_seq >= batch)) end_seq = begin_seq - 1;  // malformed
-        seq = begin_seq;
-    }
-    __device__ bool next(const DecodeParams &p, Piece &pc) {
-        while (seq <= end_seq) {
-            const int s = seq++;
-            const int n = max(p.seqlens[s], 0);
-            const int w = num_blocks_of(n);
-            const int lo = s == begin_seq ? max(begin_blk, 0) : 0;
-            const int hi = s == end_seq ? min(end_blk, w) : w;
-            if (hi <= lo) continue;
-            pc.seq = s;
-            pc.lo = lo;
-            pc.hi = hi;
-            pc.n = n;
-            pc.nsplit = p.num_splits[s + 1] - p.num_splits[s];
-            pc.slot = p.num_splits[s] + (s == begin_seq ? first_piece : 0);
-            if (pc.nsplit > 1 && (pc.slot < 0 || pc.slot >= p.batch + p.num_parts)) continue;  // malformed
-            return true;
-        }
-        return false;
-    }
-};
-
 // Walks the blocks of one part in order, with piece boundaries.
 struct BlockWalker {
     Cursor cur;
@@ -210,17 +174,13 @@ __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map
         mbar_arrive_expect_tx(&sm.kv_full[s], F8 ? kF8LoadBytes : kStageBytes);
         const int y = phys * kBlk;
         uint8_t *dst = sm.stage[s];
-        if constexpr (F8) {  // coordinates: bytes of the record (latent), bf16 elements (rotary)
-#pragma unroll
-            for (int b = 0; b < 2; ++b)
-                tma_load_2d(dst + (2 + b) * kBoxBytes, map_lat, 256 * (int)half + 128 * b, y, &sm.kv_full[s], policy);
-            tma_load_2d(dst + kRopeOffset, map_rope, 256 + 32 * (int)half, y, &sm.kv_full[s], policy);
-        } else {
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-                tma_load_2d(dst + b * kBoxBytes, map_lat, 256 * (int)half + 64 * b, y, &sm.kv_full[s], policy);
-            tma_load_2d(dst + kRopeOffset, map_rope, 512 + 32 * (int)half, y, &sm.kv_full[s], policy);
-        }
+        // the latent boxes of this half in ONE 3-D operation (an SM's TMA unit works through about one
+        // operation at a time, so few large ones keep the stream at HBM speed), then the rotary box
+        if constexpr (F8)  // coordinates: bytes of the record (latent), bf16 elements (rotary)
+            tma_load_3d(dst + 2 * kBoxBytes, map_lat, 0, y, 2 * (int)half, &sm.kv_full[s], policy);
+        else
+            tma_load_3d(dst, map_lat, 0, y, 4 * (int)half, &sm.kv_full[s], policy);
+        tma_load_2d(dst + kRopeOffset, map_rope, (F8 ? 256 : 512) + 32 * (int)half, y, &sm.kv_full[s], policy);
     }
     if (bad_block) raise_error(kErrBounds);
     // every load still in flight must land before the CTA may exit

@@ -342,3 +342,19 @@ __device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t v, u
 }
 }  // namespace sm100
 }  // namespace mla
+
+
+namespace mla {
+namespace sm100 {
+// 3-D tiled TMA load into this CTA's shared memory, completing on `bar` (transaction bytes). With
+// the cache viewed as [boxes][rows][box], one operation brings several 64-row boxes at once.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)),
+          "l"(policy) : "memory");
+}
+}  // namespace sm100
+}  // namespace mla
