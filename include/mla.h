@@ -281,9 +281,9 @@ int mla_decode_host_fp8(const void *q_host, const void *kv_cache_fp8_host, int64
  * library routine.
  *   - Returns MLA_ERR_WORKSPACE, launching nothing, when mla_workspace_bytes(batch, s_q, h_q,
  *     num_parts) exceeds MLA_NOALLOC_SCRATCH_BYTES (reduce num_parts or the batch).
- *   - The first call on each device looks up the scratch array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call before any
- *     stream capture.
+ *   - The first call on each device (and the first after a device reset, which reloads the
+ *     library's module) looks up the scratch array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
  *   - Every call on a device shares the one scratch array, which keeps the last call's
  *     contents (none of which must start at zero): calls that overlap on the GPU, e.g. on
  *     two streams, race on it and must be serialised by the caller.

@@ -17,22 +17,55 @@ constexpr size_t kNoAllocScratchBytes = (size_t)MLA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch per device. In host code the array's name is only a
-// host-side stand-in, so the address must come from cudaGetSymbolAddress, called once per
-// device with that device current.
-void *g_noalloc_ptr[kMaxDevices] = {};
+// host-side stand-in, so the address must come from cudaGetSymbolAddress, called with that device
+// current. It is cached together with the ID of the context it was looked up in: a device reset
+// (or any new primary context) reloads the module, and the next call then looks the address up
+// again instead of launching kernels on a stale one.
+struct ScratchEntry {
+    void *ptr;
+    unsigned long long ctx_id;
+};
+ScratchEntry g_noalloc[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// ID of the current context (unique for the process's lifetime), or 0 if it cannot be read.
+unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 int noalloc_scratch(void **ptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    const unsigned long long ctx = current_ctx_id();  // 0 before the runtime has made a context current
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc[dev].ptr || ctx == 0 || g_noalloc[dev].ctx_id != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        g_noalloc[dev].ptr = p;
+        g_noalloc[dev].ctx_id = current_ctx_id();  // the look-up made the device's context current
     }
-    *ptr = g_noalloc_ptr[dev];
+    *ptr = g_noalloc[dev].ptr;
     return MLA_OK;
 }
 

@@ -177,6 +177,8 @@ typedef struct {
     const uint16_t *q, *kv;
     const uint8_t *kv8; /* fp8 cache (kv == NULL), with its latent scale */
     double kv_scale;
+    double f8val[256];  /* fp8 cache: kv_scale * e4m3_to_double(code) for every code (the same values,
+                           computed once instead of once per element) */
     int64_t num_blocks;
     const int32_t *block_table;
     int64_t bt_stride;
@@ -200,7 +202,7 @@ static void load_key(const dec_job *J, int64_t row, double *k) {
         for (int d = 0; d < OR_D_QK; ++d) k[d] = bf16_bits_to_double(src[d]);
     } else {
         const uint8_t *src = J->kv8 + (size_t)row * OR_F8_REC;
-        for (int d = 0; d < OR_D_V; ++d) k[d] = J->kv_scale * e4m3_to_double(src[d]);
+        for (int d = 0; d < OR_D_V; ++d) k[d] = J->f8val[src[d]];
         for (int d = OR_D_V; d < OR_D_QK; ++d) {
             const uint8_t *r = src + OR_D_V + 2 * (d - OR_D_V); /* little-endian bf16 */
             k[d] = bf16_bits_to_double((uint16_t)(r[0] | (r[1] << 8)));
@@ -344,6 +346,8 @@ static int run_decode(const uint16_t *q, const uint16_t *kv_cache, const uint8_t
     J.bt_stride = bt_stride; J.seqlens = seqlens; J.batch = batch; J.s_q = s_q;
     J.h_q = h_q; J.causal = causal; J.scale = scale; J.out = out; J.lse = lse;
     J.tasks = tasks; J.ntasks = ntasks; J.next = 0; J.error = 0;
+    if (kv8)
+        for (int c = 0; c < 256; ++c) J.f8val[c] = kv_scale * e4m3_to_double((uint8_t)c);
     pthread_mutex_init(&J.lock, NULL);
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
     if (!th) return -2;

@@ -64,19 +64,3 @@ def full_parity(inp, num_parts=None, fixed_cost=None, what=""):
                                  inp["causal"])
     compare(bf16_to_f64(out), lse.cpu().numpy().astype(np.float64), ref_o, ref_l, what)
     return out, lse, meta
-
-
-def sample_tasks(seqlens, s_q, h_q, num_splits_cum, rng, max_rows=96):
-    """(b, t, h) rows to check at full size: the most-split, longest, shortest and random
-    sequences, several heads each, every query token."""
-    b = len(seqlens)
-    splits = np.diff(num_splits_cum)
-    seqs = {int(np.argmax(splits)), int(np.argmax(seqlens)), int(np.argmin(seqlens))}
-    one = np.nonzero(splits == 1)[0]
-    if one.size:
-        seqs.add(int(one[0]))
-    while len(seqs) < min(b, 8):
-        seqs.add(int(rng.integers(0, b)))
-    heads = sorted({0, h_q - 1} | set(int(x) for x in rng.integers(0, h_q, size=4)))
-    tasks = [(s, t, h) for s in sorted(seqs) for t in range(s_q) for h in heads]
-    return np.array(tasks[:max_rows], dtype=np.int32)

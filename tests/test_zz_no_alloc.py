@@ -3,10 +3,10 @@
 Some callers may not call cudaMalloc at decode time (a runtime with a fixed memory pool, or
 a serving path where a late allocation could fail or stall the stream). For them the library
 keeps the split partials in a fixed scratch array of its own device image instead of a
-caller workspace. These tests call that entry point through the C ABI and check that it
-returns what mla_decode returns on the same inputs, on two calls in a row (the second call
-finds the first call's leftovers in the shared scratch), with shapes whose sequences are
-split across parts so the scratch is really used.
+caller workspace. These tests call that entry point through the C ABI and check, on two calls
+in a row (the second call finds the first call's leftovers in the shared scratch), that it
+matches the CPU oracle within the parity tolerances and returns what mla_decode returns on the
+same inputs, with shapes whose sequences are split across parts so the scratch is really used.
 """
 import ctypes
 
@@ -15,6 +15,7 @@ import pytest
 import torch
 
 import mla_decode_attention_14_b200 as mla
+import oracle
 from mla_decode_attention_14_b200 import workloads as W
 from tests import parity
 
@@ -37,7 +38,7 @@ def _raw_noalloc(q, kv, bt, sl, meta, scale, causal, out, lse):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("case", CASES, ids=[str(i) for i in range(len(CASES))])
-def test_noalloc_matches_workspace_entry_point_twice(case):
+def test_noalloc_matches_oracle_and_workspace_entry_point_twice(case):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     seqlens, h_q, s_q, causal, parts = case
@@ -51,14 +52,17 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
     assert mla.check_status() == 0
     ref_o = parity.bf16_to_f64(ref_out)
     ref_l = ref_lse.cpu().numpy().astype(np.float64)
+    orc_o, orc_l = oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], wl.scale, causal)
     for call in range(2):
         out = torch.full_like(ref_out, float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
         rc = _raw_noalloc(q, kv, bt, sl, meta, wl.scale, causal, out, lse)
         assert rc == 0, mla.lib().mla_status_string(rc)
         assert mla.check_status() == 0
-        parity.compare(parity.bf16_to_f64(out), lse.cpu().numpy().astype(np.float64), ref_o, ref_l,
-                       what="noalloc call %d" % call)
+        o = parity.bf16_to_f64(out)
+        l = lse.cpu().numpy().astype(np.float64)
+        parity.compare(o, l, orc_o, orc_l, what="noalloc call %d vs oracle" % call)
+        parity.compare(o, l, ref_o, ref_l, what="noalloc call %d vs mla_decode" % call)
 
 
 @pytest.mark.gpu
