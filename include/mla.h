@@ -46,8 +46,9 @@
  *     are validated on the host BEFORE any launch;
  *     an invalid call returns a non-zero mla_status and launches nothing.
  *   - Kernels never trap. A block-table entry outside [0, num_blocks) or a pipeline
- *     wait that exceeds its iteration bound sets a per-device error word; the affected
- *     outputs are then unspecified. mla_check_status() reports and clears it.
+ *     wait that exceeds its iteration bound, or a row outside the decode's numeric range
+ *     (MLA_ERR_RANGE), sets a per-device error word; the affected outputs are then
+ *     unspecified. mla_check_status() reports and clears it.
  *   - Thread safety: calls on different streams may run concurrently; the TMA
  *     descriptor cache is guarded by a mutex.
  */
@@ -77,8 +78,9 @@ typedef enum mla_status {
     MLA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                 */
     MLA_ERR_TIMEOUT = 5,     /* a device pipeline wait hit its bound (reported by mla_check_status) */
     MLA_ERR_BOUNDS = 6,      /* a block-table entry outside [0, num_blocks) was needed */
-    MLA_ERR_RANGE = 7        /* fp8 cache: a query value outside the range of its fp16 form
-                                (reported by mla_check_status) */
+    MLA_ERR_RANGE = 7        /* a value outside the range of an internal fp16 form: an fp8-cache
+                                query value, or a row's partial-score factors (see mla_decode);
+                                reported by mla_check_status */
 } mla_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -95,9 +97,9 @@ int mla_default_num_parts(int device, int h_q, int s_q, int *num_parts);
 int mla_default_fixed_cost(int h_q, int s_q);
 
 /*
- * Bytes of device workspace mla_decode needs: fp32 partial outputs and lse for at most
- * batch + num_parts - 1 pieces of s_q*h_q rows each:
- *     (batch + num_parts) * s_q * h_q * (512 + 1) * 4, rounded up to 256.
+ * Bytes of device workspace mla_decode needs: fp32 partial outputs, lse and two precision
+ * bounds (see mla_decode) for at most batch + num_parts - 1 pieces of s_q*h_q rows each:
+ *     (batch + num_parts) * s_q * h_q * (512 + 3) * 4, rounded up to 256.
  * Returns 0 for invalid sizes. Host only.
  */
 size_t mla_workspace_bytes(int batch, int s_q, int h_q, int num_parts);
@@ -137,6 +139,15 @@ int mla_get_metadata(const int32_t *seqlens, int batch, int h_q, int s_q, int nu
  *   workspace    >= mla_workspace_bytes(batch, s_q, h_q, num_parts) bytes, 256-aligned;
  *                contents on entry are ignored
  * Requires an sm_100 device (B200). 1 <= s_q*h_q <= MLA_MAX_ROWS.
+ * Precision: the two SMs that share a row exchange, per token, the square root of its share of
+ * the softmax from their halves of q.k as fp16, relative to each SM's own partial maximum over 32
+ * tokens. That is exact to 2^-10 while a token's partial score is within ~58 octaves (about 40 in
+ * natural-log units of scale * q.k) of that maximum. A row whose dominant keys fall outside that
+ * range (its two partial maxima, from different keys, overstate its true maximum by ~50 octaves
+ * or more: far from attention at scale 192^-0.5, possible with very large scores) may lose
+ * precision in out and lse; when a bound on the error that the exchange's subnormal range adds to
+ * its softmax sum exceeds 2^-11 of the sum, the kernel sets MLA_ERR_RANGE, which mla_check_status
+ * reports. Results are then unspecified for that row.
  */
 int mla_decode(const void *q, const void *kv_cache, int64_t num_blocks,
                const int32_t *block_table, int64_t bt_stride, const int32_t *seqlens,
@@ -297,7 +308,8 @@ int mla_decode_noalloc(const void *q, const void *kv_cache, int64_t num_blocks,
 
 /*
  * Synchronises `stream`, then reads and clears this device's error word.
- * Returns MLA_OK, MLA_ERR_BOUNDS, MLA_ERR_TIMEOUT, or MLA_ERR_CUDA if a CUDA call
+ * Returns MLA_OK, MLA_ERR_BOUNDS, MLA_ERR_TIMEOUT, MLA_ERR_RANGE (in that order of priority
+ * when several bits are set), or MLA_ERR_CUDA if a CUDA call
  * (including an earlier asynchronous launch) failed.
  */
 int mla_check_status(void *stream);

@@ -17,7 +17,7 @@ cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, in
                             int32_t *tile_meta, int32_t *num_splits, cudaStream_t stream);
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q,
                            __nv_bfloat16 *out, float *lse, const float *o_part,
-                           const float *lse_part, cudaStream_t stream);
+                           const float *lse_part, const float *lost_part, cudaStream_t stream);
 cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
                                 bool fp8, cudaStream_t stream);
 cudaError_t launch_head_gemm(const CUtensorMap &map_x, const CUtensorMap &map_w, __nv_bfloat16 *y, int64_t ldy,
@@ -145,10 +145,11 @@ int shape_ok(int batch, int s_q, int h_q) {
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout: fp32 o_part[(batch + num_parts) * rows * 512], then fp32
-// lse_part[(batch + num_parts) * rows].
+// lse_part[(batch + num_parts) * rows], then fp32 lost_part[(batch + num_parts) * rows * 2].
 size_t opart_bytes(int batch, int rows, int num_parts) {
     return (size_t)(batch + num_parts) * rows * MLA_D_V * sizeof(float);
 }
+size_t lsepart_bytes(int batch, int rows, int num_parts) { return (size_t)(batch + num_parts) * rows * sizeof(float); }
 
 int validate_decode(const void *q, const void *kv, int64_t num_blocks, const int32_t *bt,
                     int64_t bt_stride, const int32_t *seqlens, const int32_t *tile_meta,
@@ -187,6 +188,8 @@ DecodeParams make_params(const void *q, const void *kv, int64_t num_blocks, cons
     p.lse = lse;
     p.o_part = static_cast<float *>(ws);
     p.lse_part = reinterpret_cast<float *>(static_cast<char *>(ws) + opart_bytes(batch, rows, num_parts));
+    p.lost_part = reinterpret_cast<float *>(static_cast<char *>(ws) + opart_bytes(batch, rows, num_parts) +
+                                            lsepart_bytes(batch, rows, num_parts));
     p.num_blocks = num_blocks;
     p.bt_stride = bt_stride;
     p.batch = batch;
@@ -247,7 +250,7 @@ int mla_default_fixed_cost(int h_q, int s_q) {
 size_t mla_workspace_bytes(int batch, int s_q, int h_q, int num_parts) {
     if (!shape_ok(batch, s_q, h_q) || num_parts < 1) return 0;
     const int rows = s_q * h_q;
-    size_t b = opart_bytes(batch, rows, num_parts) + (size_t)(batch + num_parts) * rows * sizeof(float);
+    size_t b = opart_bytes(batch, rows, num_parts) + 3 * lsepart_bytes(batch, rows, num_parts);
     return round_up(b, 256);
 }
 
@@ -339,8 +342,9 @@ int mla_decode_combine(const int32_t *num_splits, int num_parts, int batch, int 
     const float *o_part = static_cast<const float *>(workspace);
     const float *lse_part = reinterpret_cast<const float *>(static_cast<const char *>(workspace) +
                                                             opart_bytes(batch, rows, num_parts));
+    const float *lost_part = lse_part + lsepart_bytes(batch, rows, num_parts) / sizeof(float);
     cudaError_t e = launch_combine(num_splits, batch, num_parts, s_q, h_q, static_cast<__nv_bfloat16 *>(out), lse,
-                                   o_part, lse_part, static_cast<cudaStream_t>(stream));
+                                   o_part, lse_part, lost_part, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cuda_status(e);
 }

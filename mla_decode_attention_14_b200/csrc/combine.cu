@@ -8,6 +8,10 @@
 // key carry lse_s = -inf and weight 0; if every piece of a row is empty the row gets
 // out = 0, lse = -inf. Sequences with no tokens at all (no piece) are written here too.
 //
+// Each piece also leaves, per CTA half, a bound on the error that the split kernel's pair exchange
+// added to its softmax sum through fp16 subnormals, relative to that sum. The row's bound is the
+// pieces' weighted by e^{lse_s - lse}; above 2^-11 the row is reported (MLA_ERR_RANGE).
+//
 // One warp per (sequence, row); each lane owns 16 of the 512 output dims (four float4),
 // so every partial row is read as one coalesced 2 KB segment. Sequences of up to four pieces
 // (nearly all) load everything in one go; longer ones walk their pieces.
@@ -33,20 +37,27 @@ __device__ __forceinline__ void store_row(__nv_bfloat16 *orow, float *lrow, cons
 
 // Rows of sequences with 0..kFastPieces pieces: the pieces' lse and this lane's 16 dims of each
 // partial row are loaded at once, then merged from registers.
+__device__ __forceinline__ float lost_of(const float *__restrict__ lost_part, size_t slot) {
+    return fmaxf(lost_part[2 * slot], lost_part[2 * slot + 1]);  // the worse of the two CTA halves
+}
+
 __device__ __forceinline__ void combine_few(int ns, int s0, int rows, int r, int lane, __nv_bfloat16 *orow, float *lrow,
-                                            const float *__restrict__ o_part, const float *__restrict__ lse_part) {
-    float ls[kFastPieces];
+                                            const float *__restrict__ o_part, const float *__restrict__ lse_part,
+                                            const float *__restrict__ lost_part) {
+    float ls[kFastPieces], lost[kFastPieces];
     float4 v[kFastPieces][4];
 #pragma unroll
     for (int s = 0; s < kFastPieces; ++s) {
         if (s < ns) {
             const size_t slot = (size_t)(s0 + s) * rows + r;
             ls[s] = lse_part[slot];
+            lost[s] = lost_of(lost_part, slot);
             const float4 *src = reinterpret_cast<const float4 *>(o_part + slot * kDv + lane * 16);
 #pragma unroll
             for (int k = 0; k < 4; ++k) v[s][k] = src[k];
         } else {
             ls[s] = -INFINITY;
+            lost[s] = 0.f;
 #pragma unroll
             for (int k = 0; k < 4; ++k) v[s][k] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
@@ -65,10 +76,12 @@ __device__ __forceinline__ void combine_few(int ns, int s0, int rows, int r, int
 #pragma unroll
     for (int s = 0; s < kFastPieces; ++s) sum += expf(ls[s] - m);  // empty pieces: e^-inf = 0
     const float L = m + logf(sum);
+    float lost_row = 0.f;
 #pragma unroll
     for (int s = 0; s < kFastPieces; ++s) {
         const float wgt = expf(ls[s] - L);
         if (wgt == 0.f) continue;  // empty piece (its o is 0) or negligible weight
+        lost_row = fmaf(wgt, lost[s], lost_row);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             acc[4 * k + 0] += wgt * v[s][k].x;
@@ -77,13 +90,15 @@ __device__ __forceinline__ void combine_few(int ns, int s0, int rows, int r, int
             acc[4 * k + 3] += wgt * v[s][k].w;
         }
     }
+    if (lane == 0 && lost_row > 0x1p-11f) raise_error(kErrRange);
     store_row(orow, lrow, acc, L, lane);
 }
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
 combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts, int s_q, int h_q,
                __nv_bfloat16 *__restrict__ out, float *__restrict__ lse,
-               const float *__restrict__ o_part, const float *__restrict__ lse_part) {
+               const float *__restrict__ o_part, const float *__restrict__ lse_part,
+               const float *__restrict__ lost_part) {
     const int rows = s_q * h_q;
     const int b = blockIdx.x;
     const int r = blockIdx.y * kCombineWarps + (threadIdx.x >> 5);
@@ -100,7 +115,7 @@ combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts,
     __nv_bfloat16 *orow = out + ((size_t)b * rows + r) * kDv + lane * 16;
     float *lrow = lse + ((size_t)b * h_q + h) * s_q + t;
     if (ns <= kFastPieces) {  // common case: every load issued before any arithmetic (one memory round trip)
-        combine_few(ns, s0, rows, r, lane, orow, lrow, o_part, lse_part);
+        combine_few(ns, s0, rows, r, lane, orow, lrow, o_part, lse_part, lost_part);
         return;
     }
 
@@ -121,6 +136,16 @@ combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float L = m + logf(sum);
+
+    float lost_row = 0.f;
+    for (int s = lane; s < ns; s += 32) {
+        const size_t slot = (size_t)(s0 + s) * rows + r;
+        const float wgt = expf(lse_part[slot] - L);
+        if (wgt != 0.f) lost_row = fmaf(wgt, lost_of(lost_part, slot), lost_row);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lost_row += __shfl_xor_sync(0xffffffffu, lost_row, o);
+    if (lane == 0 && lost_row > 0x1p-11f) raise_error(kErrRange);
 
     float acc[16];
 #pragma unroll
@@ -144,11 +169,11 @@ combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts,
 
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q,
                            __nv_bfloat16 *out, float *lse, const float *o_part,
-                           const float *lse_part, cudaStream_t stream) {
+                           const float *lse_part, const float *lost_part, cudaStream_t stream) {
     const int rows = s_q * h_q;
     dim3 grid(batch, (rows + kCombineWarps - 1) / kCombineWarps);
     combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(num_splits, batch, num_parts, s_q, h_q, out, lse,
-                                                           o_part, lse_part);
+                                                           o_part, lse_part, lost_part);
     return cudaGetLastError();
 }
 

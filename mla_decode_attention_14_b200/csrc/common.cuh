@@ -33,6 +33,8 @@ struct DecodeParams {
     float *lse;                    // [b, h_q, s_q]
     float *o_part;                 // [slots, rows, 512]
     float *lse_part;               // [slots, rows]
+    float *lost_part;              // [slots, rows, 2]: per CTA half, a bound on the error that the pair
+                                   // exchange's subnormal range added to the piece's softmax sum, over that sum
     int64_t num_blocks;
     int64_t bt_stride;
     int batch, s_q, h_q, rows, num_parts;

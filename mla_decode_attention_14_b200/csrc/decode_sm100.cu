@@ -25,7 +25,9 @@
 //    [0, 2^15] and is normal in fp16 while s - m >= -58, so the exchange keeps a relative
 //    precision of 2^-10 (once squared) over 58 octaves of partial score whatever the score
 //    magnitude (rows whose two partial maxima overstate the true maximum by up to ~34 octaves
-//    lose nothing), and the traffic is half that of fp32 scores. The link between the two SMs
+//    lose nothing), and the traffic is half that of fp32 scores. A row that goes past that range
+//    is not lost silently: the softmax warps bound the error that subnormal peer factors add to
+//    its sum and set the range bit of the device error word when it exceeds 2^-11 of the sum. The link between the two SMs
 //    moves only about 20 bytes per cycle, so the stores are spread over the softmax warps'
 //    compute.
 //  * Eight softmax warps: warp w serves TMEM lane quarter w&3 (32 query rows) and one half of
@@ -432,7 +434,8 @@ __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &
 
 // Own partial scores of block g for this thread's 32 tokens (raw, unscaled); keys at or past `vis`
 // become -inf. The accumulators are released as soon as the scores are in registers.
-__device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&s)[kTokPer]) {
+__device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&s)[kTokPer],
+                                         int &nvalid) {
     if (!mbar_wait(&sm.s_full, g & 1, &sm.abort)) return false;
     tc_fence_after();
     {
@@ -446,6 +449,7 @@ __device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int 
     __syncwarp();
     if (c.lane == 0) mbar_arrive(&sm.s_free);
     const int k0 = key0 + kTokPer * c.th;
+    nvalid = min(max(vis - k0, 0), kTokPer);  // the valid tokens are a prefix of the thread's 32
     if (k0 + kTokPer > vis) {  // the sequence ends (or the causal limit falls) inside these tokens
 #pragma unroll
         for (int j = 0; j < kTokPer; ++j) s[j] = k0 + j < vis ? s[j] : -INFINITY;
@@ -494,6 +498,39 @@ __device__ __forceinline__ float exps_in_place(float (&s)[kTokPer], float sl2) {
     return m;
 }
 
+// Range of the exchange. A peer factor R' below 2^-14 is an fp16 subnormal (or 0) with an absolute
+// error up to 2^-25, i.e. a relative error up to 2^-25 / R' where a normal one has 2^-11. The part of
+// its token's P = (R_own R' fh)^2 past normal precision is then at most R_own^2 fh^2 R' (2^-24 -
+// 2^-10 R') = P (2^-24 / R' - 2^-10), and R_own^2 fh^2 2^-50 <= fh^2 2^-20 when R' = 0 (R_own <=
+// 2^15). Non-negative fp16 numbers order like their bit patterns, so the u16x2 minimum of a thread's
+// 32 factors (`mn`, per token parity) shows whether any is below 2^-14 (valid tokens of rows whose
+// partial maxima overstate the true maximum by ~58 octaves or more; masked tokens carry R' = 0).
+// Only then is the bound summed (the warp votes, so that it branches once).
+// The bound above for tokens 8 c4 .. 8 c4 + 7 of this thread (those below `nv` are valid), in units
+// of l. `w4`: their peer factors (fp16 pairs); `pk`/`pl`: P as stored for Gemm2 (bf16 hi/lo pairs;
+// fp8 cache: fp16 pairs in `pk`).
+template <bool F8>
+__device__ __forceinline__ float range_excess8(const uint32_t (&w4)[4], int c4, const uint32_t (&pk)[kTokPer / 2],
+                                               const uint32_t (&pl)[kTokPer / 2], int nv, float fh) {
+    float sq = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int j = 8 * c4 + k, sh = 16 * (k & 1);
+        const uint32_t hb = (w4[k >> 1] >> sh) & 0xffffu;
+        if (hb >= 0x400u || j >= nv) continue;  // normal, or a masked token
+        const float rp = __half2float(__ushort_as_half((unsigned short)hb));
+        float pj;
+        if constexpr (F8) {
+            pj = __half2float(__ushort_as_half((unsigned short)(pk[j >> 1] >> sh)));
+        } else {  // hi + lo, each a bf16 (the top half of an fp32)
+            pj = __uint_as_float(((pk[j >> 1] >> sh) & 0xffffu) << 16) +
+                 __uint_as_float(((pl[j >> 1] >> sh) & 0xffffu) << 16);
+        }
+        sq += rp > 0.f ? pj * (0x1p-24f / rp - 0x1p-10f) : 0x1p-20f * fh * fh;
+    }
+    return sq;
+}
+
 template <bool F8>
 __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem, uint32_t half,
                              int group) {
@@ -530,7 +567,8 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     load_q<F8>(sm, c, w.pc);
     int vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
     float e_own[kTokPer], m_own;
-    if (!load_raw(sm, c, 0, w.blk * kBlk, vis, e_own)) return;
+    int nv_own;  // valid tokens of the block being finished, among this thread's 32
+    if (!load_raw(sm, c, 0, w.blk * kBlk, vis, e_own, nv_own)) return;
     m_own = exps_in_place(e_own, sl2);
     send_factors(c, 0, e_own, m_own);
     if (w.last()) {  // the next piece's Q may replace this one once its last Gemm1 is done
@@ -539,6 +577,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         if (tmp.next(p, nx)) load_q<F8>(sm, c, nx);
     }
     float m_ref = -INFINITY, l = 0.f;
+    float lost = 0.f;  // bound on the part of l past normal precision from subnormal peer factors (scale of l)
     for (int g = 0; w.live; ++g) {
         const bool a_first = w.first(), a_last = w.last();
         const int a_piece_k = w.piece_k, a_seq = w.pc.seq, a_nsplit = w.pc.nsplit, a_slot = w.pc.slot;
@@ -547,9 +586,10 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         // raw scores of block g+1 first: the accumulators are free for Gemm1 of block g+2 early, and
         // the peer's factors of block g arrive meanwhile
         float snx[kTokPer];
+        int nv_nx = 0;
         if (nx_live) {
             if (w.first()) vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
-            if (!load_raw(sm, c, g + 1, w.blk * kBlk, vis, snx)) return;
+            if (!load_raw(sm, c, g + 1, w.blk * kBlk, vis, snx, nv_nx)) return;
             if (w.last()) {
                 Cursor tmp = w.cur;
                 Piece nx;
@@ -566,6 +606,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         const float m_peer = c.warp_ok ? xo[(slot * kTq + c.th) * 128 + c.i] : -INFINITY;
         const float mbu_half = m_own + m_peer;
         uint32_t ep[kTokPer / 2];  // the peer's factors, fp16 pairs
+        uint32_t mn = 0xffffffffu;  // their minimum per token parity (non-negative fp16 order like their bits)
         float mbu;                 // the block's row max (both token halves), shared by the two warps of a row
         if constexpr (F8) {
             // exact: t_j = R_own R_peer = 2^((s_j - m_own - m_peer) / 2 + 30) in place of R_own, and
@@ -601,6 +642,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         if (a_first) {
             m_ref = mbu;
             l = 0.f;
+            lost = 0.f;
         } else if (mbu > m_ref + kRescaleThreshold) {
             if (m_ref == -INFINITY) {
                 m_ref = mbu;  // nothing accumulated yet (O and l are zero)
@@ -608,6 +650,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 alpha = ex2_approx(m_ref - mbu);
                 m_ref = mbu;
                 l *= alpha;
+                lost *= alpha;
                 need = true;
             }
         }
@@ -628,8 +671,13 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         // slot (g - 1) % 2 = (g + 1) % 2.
         // P = 2^(s0 + s1 - m_ref) in two bf16 terms: hi = P with its low 16 bits cleared, lo = the
         // (exact) remainder with its low 16 bits cleared; hi + lo is within 2^-14 of P.
+        // P = (t fh)^2 with t = R_own R_peer and fh = 2^((mbu_half - m_ref) / 2 - 30), the square root
+        // of the block's factor: fh stays a normal fp32 number down to mbu_half - m_ref = -192, where P
+        // itself is below 2^-126, so no block that can matter is flushed. The exponent is capped at 64,
+        // reached only when the fp8 path's exact row max lies more than ~190 octaves below the sum of
+        // the partial maxima (a row the range check below reports).
         const bool none = m_ref == -INFINITY || mbu_half == -INFINITY;
-        const float f = none ? 0.f : ex2_approx(mbu_half - m_ref - 4.f * kXScaleLog2);
+        const float fh = none ? 0.f : ex2_approx(fminf(0.5f * (mbu_half - m_ref) - 2.f * kXScaleLog2, 64.f));
         float m_nx, off_nx;
         {
             const float smax = max32(snx);
@@ -645,7 +693,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         // instruction, each rounded as its scalar form would be).
         uint32_t pk[kTokPer / 2], pl[kTokPer / 2];
         f32x2 su[4] = {0ull, 0ull, 0ull, 0ull};  // two lanes of partial row sums each (0 is +0, +0)
-        const f32x2 ff = pack2(f, f), hsl2 = pack2(0.5f * sl2, 0.5f * sl2), offnx = pack2(off_nx, off_nx);
+        const f32x2 ffh = pack2(fh, fh), hsl2 = pack2(0.5f * sl2, 0.5f * sl2), offnx = pack2(off_nx, off_nx);
         const f32x2 minus1 = pack2(-1.f, -1.f);
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
@@ -660,10 +708,11 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 snx[j + 1] = ex2_approx(x1);
                 __half2 two = __floats2half2_rn(snx[j], snx[j + 1]);
                 wv[q] = *reinterpret_cast<uint32_t *>(&two);
+                mn = min_u16x2(mn, ep[j >> 1]);
                 // P of block g
                 if constexpr (F8) {  // e_own holds t = R_own R_peer; P in fp16 (round to nearest)
-                    const f32x2 t = pack2(e_own[j], e_own[j + 1]);
-                    const f32x2 pp = mul2(mul2(t, t), ff);
+                    const f32x2 tf = mul2(pack2(e_own[j], e_own[j + 1]), ffh);
+                    const f32x2 pp = mul2(tf, tf);
                     su[q] = add2(su[q], pp);
                     float p0, p1;
                     unpack2(pp, p0, p1);
@@ -671,8 +720,8 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                     pk[j >> 1] = *reinterpret_cast<uint32_t *>(&ph);
                 } else {
                     const float2 e2 = __half22float2(*reinterpret_cast<const __half2 *>(&ep[j >> 1]));
-                    const f32x2 t = mul2(pack2(e_own[j], e_own[j + 1]), pack2(e2.x, e2.y));
-                    const f32x2 pp = mul2(mul2(t, t), ff);
+                    const f32x2 tf = mul2(mul2(pack2(e_own[j], e_own[j + 1]), pack2(e2.x, e2.y)), ffh);
+                    const f32x2 pp = mul2(tf, tf);
                     su[q] = add2(su[q], pp);
                     float p0, p1;
                     unpack2(pp, p0, p1);
@@ -686,6 +735,22 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 }
             }
             if (send) st_async_v4_b32(xbase + c4 * 128 * 16, wv[0], wv[1], wv[2], wv[3], xbar);
+        }
+        // Range of the exchange (see range_excess8). bf16 cache: the bound is summed here, with R'
+        // read again from the receive slot 16 bytes at a time (the peer refills that slot only after
+        // it has the row offset of block g+1, sent below), so the factors need not stay in registers.
+        const bool suspect = fh > 0.f && ((mn & 0xffffu) < 0x400u || (mn >> 16) < 0x400u);
+        if constexpr (!F8) {
+            if (__any_sync(0xffffffffu, suspect) && suspect) {
+                float sq = 0.f;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint4 v = xe[((slot * kTq + c.th) * 4 + c4) * 128 + c.i];
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                    sq += range_excess8<F8>(w4, c4, pk, pl, nv_own, fh);
+                }
+                lost += sq;
+            }
         }
         if (send)  // the row offset travels in the offsets area of the same slot
             st_async_b32(xchg_peer + (uint32_t)kXchgEBytes + (uint32_t)((nslot * kTq + c.th) * 128 + c.i) * 4,
@@ -718,13 +783,38 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         tc_fence_before();
         __syncwarp();
         if (c.lane == 0) mbar_arrive(&sm.p_full);
+        // fp8 cache: the range bound once Gemm2 has its operand, from the factors still in registers
+        if constexpr (F8) {
+            if (__any_sync(0xffffffffu, suspect) && suspect) {
+                float sq = 0.f;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint32_t w4[4] = {ep[4 * c4], ep[4 * c4 + 1], ep[4 * c4 + 2], ep[4 * c4 + 3]};
+                    sq += range_excess8<F8>(w4, c4, pk, pl, nv_own, fh);
+                }
+                lost += sq;
+            }
+        }
 
         if (a_last) {  // epilogue of this piece: the two token halves' sums, then this warp's O columns
-            // the sums travel in the other parity's row-max slots, which nobody reads until block g+1
+            // the sums travel in the other parity's row-max slots, which nobody reads until block g+1,
+            // the loss bounds in this parity's, which both warps of the row have read by now
             sm.xmax[(g + 1) & 1][c.th][c.i] = l;
+            sm.xmax[g & 1][c.th][c.i] = lost;
             named_bar_sync(bar_id, 64);
             const float l_row = l + sm.xmax[(g + 1) & 1][c.th ^ 1][c.i];
+            const float lost_row = lost + sm.xmax[g & 1][c.th ^ 1][c.i];
             named_bar_sync(bar_id, 64);  // both sums read before block g+1 reuses the slots
+            // Range of the exchange: a whole row is reported here when the bound exceeds 2^-11 of its
+            // sum; a piece leaves bound / sum for the combine, which weighs the pieces of the row.
+            if (c.row_ok && c.th == 0) {
+                if (a_nsplit == 1 || !(l_row > 0.f)) {
+                    if (lost_row > 0x1p-11f * l_row) raise_error(kErrRange);
+                    if (a_nsplit != 1) p.lost_part[((size_t)a_slot * p.rows + c.r) * 2 + half] = 0.f;
+                } else {
+                    p.lost_part[((size_t)a_slot * p.rows + c.r) * 2 + half] = lost_row / l_row;
+                }
+            }
             if (!mbar_wait(&sm.o_full, a_piece_k & 1, abort)) return;
             tc_fence_after();
             if (c.warp_ok) {
@@ -779,6 +869,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
 #pragma unroll
             for (int j = 0; j < kTokPer; ++j) e_own[j] = snx[j];
             m_own = m_nx;
+            nv_own = nv_nx;
         }
     }
 }

@@ -50,7 +50,7 @@ def test_status_strings(L):
 
 def test_workspace_formula(L):
     b, s_q, h_q, P = 128, 1, 128, 74
-    raw = (b + P) * s_q * h_q * (512 + 1) * 4
+    raw = (b + P) * s_q * h_q * (512 + 3) * 4
     assert L.mla_workspace_bytes(b, s_q, h_q, P) == (raw + 255) // 256 * 256
     assert L.mla_workspace_bytes(0, 1, 1, 1) == 0
     assert L.mla_workspace_bytes(1, 1, 2000, 1) == 0   # rows above MLA_MAX_ROWS
