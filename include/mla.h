@@ -202,6 +202,35 @@ int mla_decode_split_fp8(const void *q, const void *kv_cache_fp8, int64_t num_bl
                          float *lse, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Sparse decode over the bf16 cache: every query token attends to a list of cache positions
+ * instead of its whole sequence. The pages recommend a sparse attention mode for sequences over 8K
+ * tokens ("Playing DeepSeek on the cloud, part 5: ... FlashMLA accelerating DeepSeek-V2-Lite
+ * inference", section 4 "developer practice", item 2 "monitoring and tuning") without saying what is
+ * sparse; this library's reading: row (b, t, h) attends only to the keys at the positions
+ * indices[b, t, 0..topk), shared by the h_q heads of that token.
+ *   indices   int32[batch, s_q, topk], 4-byte aligned: positions within sequence b. An entry outside
+ *             [0, seqlens[b]) is no key (e.g. -1 padding); an entry listed twice counts twice; order
+ *             does not matter. No causal mask applies (the list decides). A row with no key gets
+ *             out = 0, lse = -inf.
+ *   topk      1 <= topk <= 2^24
+ *   tile_meta, num_splits, num_parts: from mla_get_metadata_sparse with the same batch, s_q, h_q,
+ *             topk (the work units are the batch * s_q query tokens, each with topk keys)
+ *   workspace >= mla_workspace_bytes(batch * s_q, 1, h_q, num_parts) bytes, 256-aligned
+ * All other arguments, outputs, precision and status rules are those of mla_decode (q, out and lse
+ * have the same shapes; 1 <= batch * s_q <= MLA_MAX_BATCH, 1 <= h_q <= MLA_MAX_ROWS). A position whose
+ * block-table entry lies outside [0, num_blocks) (or past bt_stride) is treated as no key and
+ * reported as MLA_ERR_BOUNDS by mla_check_status. Launches the split and combine kernels on
+ * `stream`; allocates nothing.
+ */
+int mla_get_metadata_sparse(int batch, int s_q, int h_q, int topk, int num_parts, int fixed_cost,
+                            int32_t *tile_meta, int32_t *num_splits, void *stream);
+int mla_decode_sparse(const void *q, const void *kv_cache, int64_t num_blocks, const int32_t *block_table,
+                      int64_t bt_stride, const int32_t *seqlens, const int32_t *indices, int topk,
+                      const int32_t *tile_meta, const int32_t *num_splits, int num_parts, int batch, int s_q,
+                      int h_q, float scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                      void *stream);
+
+/*
  * Appending new tokens to the paged cache, the step that precedes decode. Token t of sequence b's
  * new tokens goes to position p = seqlens[b] + t of that sequence, i.e. cache row
  * block_table[b][p / 64] * 64 + p % 64 ("Deep analysis of the DeepSeek Infra open-source releases",

@@ -40,7 +40,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # exported C symbols, in the order include/mla.h declares them
 EXPORTS = ("mla_status_string", "mla_default_num_parts", "mla_default_fixed_cost", "mla_workspace_bytes",
            "mla_get_metadata", "mla_decode", "mla_decode_split", "mla_decode_combine", "mla_decode_fp8",
-           "mla_decode_split_fp8", "mla_append_kv", "mla_append_kv_fp8", "mla_head_gemm",
+           "mla_decode_split_fp8", "mla_get_metadata_sparse", "mla_decode_sparse", "mla_append_kv", "mla_append_kv_fp8", "mla_head_gemm",
            "mla_decode_host", "mla_decode_host_fp8",
            "mla_decode_noalloc", "mla_check_status", "mla_launch_count", "mla_last_cuda_error",
            "mla_selftest_wait_timeout")
@@ -89,6 +89,10 @@ def lib():
         for name in ("mla_decode_fp8", "mla_decode_split_fp8"):
             getattr(L, name).argtypes = dec8
             getattr(L, name).restype = I
+        L.mla_get_metadata_sparse.argtypes = [I, I, I, I, I, I, P, P, P]
+        L.mla_get_metadata_sparse.restype = I
+        L.mla_decode_sparse.argtypes = [P, P, I64, P, I64, P, P, I, P, P, I, I, I, I, F, P, P, P, SZ, P]
+        L.mla_decode_sparse.restype = I
         L.mla_append_kv.argtypes = [P, I, P, I64, P, I64, P, I, P]
         L.mla_append_kv.restype = I
         L.mla_append_kv_fp8.argtypes = [P, I, P, I64, F, P, I64, P, I, P]
@@ -149,6 +153,7 @@ class Metadata:
     fixed_cost: int
     h_q: int
     s_q: int
+    topk: int = 0             # sparse mode (get_metadata_sparse): keys per query token; 0 = dense
 
 
 def default_num_parts(h_q: int, s_q: int, device=None) -> int:
@@ -181,6 +186,64 @@ def get_metadata(seqlens: torch.Tensor, h_q: int, s_q: int, num_parts: int | Non
         _check("mla_get_metadata", lib().mla_get_metadata(seqlens.data_ptr(), b, h_q, s_q, num_parts, fixed_cost,
                                                           tm.data_ptr(), ns.data_ptr(), _stream(stream)))
     return Metadata(tm, ns, num_parts, fixed_cost, h_q, s_q)
+
+
+def get_metadata_sparse(batch: int, s_q: int, h_q: int, topk: int, num_parts: int | None = None,
+                        fixed_cost: int | None = None, device=None, stream=None) -> Metadata:
+    """Schedule for :func:`decode_sparse`: ``batch * s_q`` work units (one per query token) of
+    ``topk`` keys each (``mla_get_metadata_sparse``)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if num_parts is None:
+        num_parts = default_num_parts(h_q, 1, dev)
+    if fixed_cost is None:
+        fixed_cost = default_fixed_cost(h_q, 1)
+    tm = torch.empty((num_parts, META_INTS), dtype=torch.int32, device=dev)
+    ns = torch.empty((batch * s_q + 1,), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check("mla_get_metadata_sparse", lib().mla_get_metadata_sparse(batch, s_q, h_q, topk, num_parts, fixed_cost,
+                                                                        tm.data_ptr(), ns.data_ptr(),
+                                                                        _stream(stream)))
+    return Metadata(tm, ns, num_parts, fixed_cost, h_q, s_q, topk)
+
+
+def decode_sparse(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+                  indices: torch.Tensor, scale: float, meta: Metadata, out: torch.Tensor | None = None,
+                  lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """Sparse MLA decode (``mla_decode_sparse``): row (b, t, h) attends only to the cache positions
+    ``indices[b, t, :]`` (int32 ``[b, s_q, topk]``; entries outside ``[0, seqlens[b])`` are no key).
+    Returns ``(out bf16 [b, s_q, h_q, 512], lse fp32 [b, h_q, s_q])``."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(kv_cache, "kv_cache", torch.bfloat16)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    _need(indices, "indices", torch.int32, 3)
+    b, s_q, h_q, d = q.shape
+    topk = indices.shape[2]
+    if d != D_QK or kv_cache.shape[-1] != D_QK or kv_cache.shape[1] != BLOCK:
+        raise ValueError("q must be [b, s_q, h_q, 576] and kv_cache [num_blocks, 64, 1, 576]")
+    if block_table.shape[0] != b or seqlens.shape[0] != b or indices.shape[:2] != (b, s_q):
+        raise ValueError("batch mismatch between q, block_table, seqlens and indices")
+    if meta.topk != topk or meta.h_q != h_q or meta.s_q != s_q or meta.num_splits.shape[0] != b * s_q + 1:
+        raise ValueError("metadata was computed for another shape (use get_metadata_sparse)")
+    dev = q.device
+    if out is None:
+        out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    ws_bytes = workspace_bytes(b * s_q, 1, h_q, meta.num_parts)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    if workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError("workspace too small: need %d bytes" % ws_bytes)
+    with torch.cuda.device(dev):
+        _check("mla_decode_sparse", lib().mla_decode_sparse(
+            q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(), block_table.shape[1],
+            seqlens.data_ptr(), indices.data_ptr(), topk, meta.tile_meta.data_ptr(), meta.num_splits.data_ptr(),
+            meta.num_parts, b, s_q, h_q, float(scale), out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+            ws_bytes, _stream(stream)))
+    return out, lse
 
 
 def _decode_args(q, kv_cache, block_table, seqlens, meta):

@@ -13,9 +13,9 @@
 
 namespace mla {
 
-cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, int fixed_cost,
+cudaError_t launch_metadata(const int32_t *seqlens, int uniform_n, int batch, int num_parts, int fixed_cost,
                             int32_t *tile_meta, int32_t *num_splits, cudaStream_t stream);
-cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q,
+cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q, int sp_sq,
                            __nv_bfloat16 *out, float *lse, const float *o_part,
                            const float *lse_part, const float *lost_part, cudaStream_t stream);
 cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
@@ -142,6 +142,13 @@ int shape_ok(int batch, int s_q, int h_q) {
     return 1;
 }
 
+// Sparse mode: batch * s_q work units of h_q rows each (every row of a unit shares its index list).
+int sparse_shape_ok(int batch, int s_q, int h_q, int topk) {
+    if (batch < 1 || s_q < 1 || h_q < 1 || topk < 1 || topk > (1 << 24)) return 0;
+    if ((int64_t)batch * s_q > (1 << 24)) return 0;
+    return shape_ok(batch * s_q, 1, h_q);
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout: fp32 o_part[(batch + num_parts) * rows * 512], then fp32
@@ -203,6 +210,9 @@ DecodeParams make_params(const void *q, const void *kv, int64_t num_blocks, cons
     p.v_scale = 1.f;
     p.q_lat_mul = 1.f;
     p.q_rope_mul = 1.f;
+    p.indices = nullptr;  // dense
+    p.topk = 0;
+    p.sp_sq = 0;
     return p;
 }
 
@@ -263,7 +273,7 @@ int mla_get_metadata(const int32_t *seqlens, int batch, int h_q, int s_q, int nu
     if (!aligned(seqlens, 4) || !aligned(tile_meta, 4) || !aligned(num_splits, 4)) return MLA_ERR_INVALID_ARG;
     int rc = check_device();
     if (rc != MLA_OK) return rc;
-    cudaError_t e = launch_metadata(seqlens, batch, num_parts, fixed_cost, tile_meta, num_splits,
+    cudaError_t e = launch_metadata(seqlens, 0, batch, num_parts, fixed_cost, tile_meta, num_splits,
                                     static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cuda_status(e);
@@ -343,8 +353,8 @@ int mla_decode_combine(const int32_t *num_splits, int num_parts, int batch, int 
     const float *lse_part = reinterpret_cast<const float *>(static_cast<const char *>(workspace) +
                                                             opart_bytes(batch, rows, num_parts));
     const float *lost_part = lse_part + lsepart_bytes(batch, rows, num_parts) / sizeof(float);
-    cudaError_t e = launch_combine(num_splits, batch, num_parts, s_q, h_q, static_cast<__nv_bfloat16 *>(out), lse,
-                                   o_part, lse_part, lost_part, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_combine(num_splits, batch, num_parts, s_q, h_q, 0, static_cast<__nv_bfloat16 *>(out),
+                                   lse, o_part, lse_part, lost_part, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cuda_status(e);
 }
@@ -373,6 +383,53 @@ int mla_decode_fp8(const void *q, const void *kv_cache_fp8, int64_t num_blocks, 
     if (rc != MLA_OK) return rc;
     return mla_decode_combine(num_splits, num_parts, batch, s_q, h_q, out, lse, workspace,
                               workspace_bytes, stream);
+}
+
+int mla_get_metadata_sparse(int batch, int s_q, int h_q, int topk, int num_parts, int fixed_cost,
+                            int32_t *tile_meta, int32_t *num_splits, void *stream) {
+    if (!tile_meta || !num_splits) return MLA_ERR_INVALID_ARG;
+    if (!sparse_shape_ok(batch, s_q, h_q, topk) || num_parts < 1 || num_parts > 65535 || fixed_cost < 0 ||
+        fixed_cost > (1 << 20))
+        return MLA_ERR_INVALID_ARG;
+    if (!aligned(tile_meta, 4) || !aligned(num_splits, 4)) return MLA_ERR_INVALID_ARG;
+    int rc = check_device();
+    if (rc != MLA_OK) return rc;
+    cudaError_t e = launch_metadata(nullptr, topk, batch * s_q, num_parts, fixed_cost, tile_meta, num_splits,
+                                    static_cast<cudaStream_t>(stream));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_status(e);
+}
+
+int mla_decode_sparse(const void *q, const void *kv_cache, int64_t num_blocks, const int32_t *block_table,
+                      int64_t bt_stride, const int32_t *seqlens, const int32_t *indices, int topk,
+                      const int32_t *tile_meta, const int32_t *num_splits, int num_parts, int batch, int s_q,
+                      int h_q, float scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+    if (!indices || !aligned(indices, 4)) return MLA_ERR_INVALID_ARG;
+    if (!sparse_shape_ok(batch, s_q, h_q, topk)) return MLA_ERR_INVALID_ARG;
+    const int units = batch * s_q;  // one work unit per (sequence, query token), s_q = 1 each
+    // the dense checks with the work-unit shape; seqlens has `batch` entries, read only by the kernel
+    int rc = validate_decode(q, kv_cache, num_blocks, block_table, bt_stride, seqlens, tile_meta, num_splits,
+                             num_parts, units, 1, h_q, scale, 0, out, lse, workspace, workspace_bytes);
+    if (rc != MLA_OK) return rc;
+    rc = check_device();
+    if (rc != MLA_OK) return rc;
+    DecodeParams p = make_params(q, kv_cache, num_blocks, block_table, bt_stride, seqlens, tile_meta, num_splits,
+                                 num_parts, units, 1, h_q, scale, 0, out, lse, workspace);
+    p.indices = indices;
+    p.topk = topk;
+    p.sp_sq = s_q;
+    CUtensorMap unused;
+    std::memset(&unused, 0, sizeof(unused));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_decode_sm100(p, unused, unused, false, st);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return cuda_status(e);
+    const float *lost_part = p.lse_part + lsepart_bytes(units, h_q, num_parts) / sizeof(float);
+    e = launch_combine(num_splits, units, num_parts, 1, h_q, s_q, static_cast<__nv_bfloat16 *>(out), lse, p.o_part,
+                       p.lse_part, lost_part, st);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_status(e);
 }
 
 static int append_common(const void *new_kv, int n_new, void *kv, int64_t num_blocks, const int32_t *block_table,

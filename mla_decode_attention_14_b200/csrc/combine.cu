@@ -95,7 +95,7 @@ __device__ __forceinline__ void combine_few(int ns, int s0, int rows, int r, int
 }
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
-combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts, int s_q, int h_q,
+combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts, int s_q, int h_q, int sp_sq,
                __nv_bfloat16 *__restrict__ out, float *__restrict__ lse,
                const float *__restrict__ o_part, const float *__restrict__ lse_part,
                const float *__restrict__ lost_part) {
@@ -113,7 +113,9 @@ combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts,
     }
     const int t = r / h_q, h = r % h_q;
     __nv_bfloat16 *orow = out + ((size_t)b * rows + r) * kDv + lane * 16;
-    float *lrow = lse + ((size_t)b * h_q + h) * s_q + t;
+    // sparse mode (sp_sq > 0): work unit b is query token b % sp_sq of sequence b / sp_sq
+    float *lrow = sp_sq > 0 ? lse + ((size_t)(b / sp_sq) * h_q + h) * sp_sq + b % sp_sq
+                            : lse + ((size_t)b * h_q + h) * s_q + t;
     if (ns <= kFastPieces) {  // common case: every load issued before any arithmetic (one memory round trip)
         combine_few(ns, s0, rows, r, lane, orow, lrow, o_part, lse_part, lost_part);
         return;
@@ -167,12 +169,12 @@ combine_kernel(const int32_t *__restrict__ num_splits, int batch, int num_parts,
     store_row(orow, lrow, acc, L, lane);
 }
 
-cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q,
+cudaError_t launch_combine(const int32_t *num_splits, int batch, int num_parts, int s_q, int h_q, int sp_sq,
                            __nv_bfloat16 *out, float *lse, const float *o_part,
                            const float *lse_part, const float *lost_part, cudaStream_t stream) {
     const int rows = s_q * h_q;
     dim3 grid(batch, (rows + kCombineWarps - 1) / kCombineWarps);
-    combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(num_splits, batch, num_parts, s_q, h_q, out, lse,
+    combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(num_splits, batch, num_parts, s_q, h_q, sp_sq, out, lse,
                                                            o_part, lse_part, lost_part);
     return cudaGetLastError();
 }

@@ -35,6 +35,11 @@ struct DecodeParams {
     float *lse_part;               // [slots, rows]
     float *lost_part;              // [slots, rows, 2]: per CTA half, a bound on the error that the pair
                                    // exchange's subnormal range added to the piece's softmax sum, over that sum
+    // sparse mode: work unit (sequence) u is query token u % sp_sq of sequence u / sp_sq, with s_q = 1
+    // and causal = 0; its keys are the cache positions indices[u, 0..topk) (entries outside
+    // [0, seqlens[u / sp_sq]) are no key)
+    const int32_t *indices;        // [b * sp_sq, topk], or null (dense)
+    int topk, sp_sq;
     int64_t num_blocks;
     int64_t bt_stride;
     int batch, s_q, h_q, rows, num_parts;

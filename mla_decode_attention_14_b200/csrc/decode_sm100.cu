@@ -119,6 +119,7 @@ struct __align__(1024) Smem {
     uint8_t q_rope[128 * 64];             // rotary query dims [128 rows x 32], K-major, 64-byte swizzle
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t conv_full[kStages];  // fp8 cache: the stage's latent is in fp16
+    uint64_t vmask[kStages];      // sparse mode: bit j = token j of the stage is a key
     uint64_t s_full, s_free, p_full, p_free, o_full, o_free, q_full, mma_done;
     uint64_t xfull[2];  // receive slots filled by the peer
     uint32_t tmem_base;
@@ -127,9 +128,10 @@ struct __align__(1024) Smem {
 
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory (with 1 KB for alignment) must fit 227 KB");
 
-// Walks the blocks of one part in order, with piece boundaries.
+// Walks the blocks of one part in order, with piece boundaries (SP: sparse mode).
+template <bool SP = false>
 struct BlockWalker {
-    Cursor cur;
+    Cursor<SP> cur;
     Piece pc;
     int blk, piece_k;
     bool live;
@@ -160,7 +162,7 @@ template <bool F8>
 __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map_lat, const CUtensorMap *map_rope,
                          const int32_t *meta, uint32_t half) {
     const uint64_t policy = l2_evict_first_policy();
-    BlockWalker w;
+    BlockWalker<> w;
     w.init(meta, p);
     int gidx = 0;
     bool bad_block = false;
@@ -193,12 +195,77 @@ __device__ void producer(Smem &sm, const DecodeParams &p, const CUtensorMap *map
     }
 }
 
-// ---------------------------------------------------------------- MMA issuing warps
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int lane) {
     bool ok = true;
     if (lane == 0) ok = mbar_wait(bar, parity, abort);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
+
+// ---------------------------------------------------------------- sparse mode: gather producer (1 warp)
+// Block k of work unit u holds the keys listed at indices[u, 64k .. 64k+64). Lane l resolves
+// entries l and l + 32: a position inside [0, seqlens[b]) is a key, read from cache row
+// block_table[b, pos / 64] * 64 + pos % 64; anything else (or a list shorter than the block) is no
+// key, copied as zeros. Then, token by token, the 32 lanes copy this CTA's 512-byte latent half of
+// the row, one 16-byte chunk each (one coalesced 512-byte read), and lanes 0-3 its 64-byte rotary
+// half, with 16-byte asynchronous copies into the positions the stage's 128-byte (latent) and
+// 64-byte (rotary) swizzles give them -- the layout the MMA descriptors read, which a TMA box cannot
+// produce for single rows. The stage's validity mask is stored before lane 0's arrival on kv_full;
+// each lane's copies complete on kv_full too (33 arrivals per fill).
+__device__ void gather_producer(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t half) {
+    const int lane = threadIdx.x & 31;
+    volatile int *abort = &sm.abort;
+    const char *kv = reinterpret_cast<const char *>(p.kv);
+    BlockWalker<true> w;
+    w.init(meta, p);
+    int gidx = 0;
+    bool bad_entry = false;
+    for (; w.live; w.advance(p), ++gidx) {
+        const int s = gidx % kStages, fill = gidx / kStages;
+        if (fill > 0 && !warp_wait(&sm.kv_empty[s], (fill - 1) & 1, abort, lane)) break;
+        const int b = w.pc.seq / p.sp_sq;
+        const int n = max(__ldg(&p.seqlens[b]), 0);
+        const int32_t *list = p.indices + (size_t)w.pc.seq * p.topk;
+        int row[2];  // cache row (physical block * 64 + slot) of entries lane and lane + 32, or -1
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = w.blk * kBlk + 32 * u + lane;
+            const int pos = e < p.topk ? __ldg(&list[e]) : -1;
+            row[u] = -1;
+            if (pos >= 0 && pos < n) {
+                const int blk = pos / kBlk;
+                const int phys = blk < p.bt_stride ? __ldg(&p.block_table[(size_t)b * p.bt_stride + blk]) : -1;
+                if (phys >= 0 && (int64_t)phys < p.num_blocks)
+                    row[u] = phys * kBlk + pos % kBlk;
+                else
+                    bad_entry = true;  // reported; the entry is treated as no key
+            }
+        }
+        const uint64_t mask = (uint64_t)__ballot_sync(0xffffffffu, row[0] >= 0) |
+                              ((uint64_t)__ballot_sync(0xffffffffu, row[1] >= 0) << 32);
+        const uint32_t dst = smem_addr(sm.stage[s]);
+#pragma unroll 4
+        for (int t = 0; t < kBlk; ++t) {
+            const int r = __shfl_sync(0xffffffffu, t < 32 ? row[0] : row[1], t & 31);
+            const uint32_t bytes = r >= 0 ? 16u : 0u;  // 0: the chunk is zero-filled, nothing is read
+            const char *src = kv + (size_t)(r >= 0 ? r : 0) * (kDqk * 2);
+            // latent chunk `lane` of this half: dims 256 half + 8 lane, box lane / 8, chunk lane % 8
+            cp_async_16(dst + (lane >> 3) * kBoxBytes + t * 128 + (((lane & 7) ^ (t & 7)) << 4),
+                        src + (256 * half + 8 * lane) * 2, bytes);
+            if (lane < 4)  // rotary chunk `lane`: dims 512 + 32 half + 8 lane (64-byte swizzle)
+                cp_async_16(dst + kRopeOffset + t * 64 + ((lane ^ ((t >> 1) & 3)) << 4),
+                            src + (512 + 32 * half + 8 * lane) * 2, bytes);
+        }
+        if (lane == 0) {
+            sm.vmask[s] = mask;
+            mbar_arrive(&sm.kv_full[s]);
+        }
+        cp_async_mbar_arrive_noinc(&sm.kv_full[s]);
+    }
+    if (bad_entry) raise_error(kErrBounds);
+    cp_async_wait_all();  // every copy lands before the CTA may exit
+}
+
+// ---------------------------------------------------------------- MMA issuing warps
 
 // Zero the cache rows past a sequence's end in its last block (undefined contents -- possibly
 // NaN -- must not reach Gemm2 even with zero probabilities).
@@ -240,7 +307,7 @@ __device__ void convert_warp(Smem &sm, const DecodeParams &p, const int32_t *met
     const int u = lane & 7, hp = (lane >> 3) & 1, pq = lane >> 4;  // chunk, half of the pair, pair of the step
     const int k0 = 2 * (u & 3);                                     // first fp16 chunk of the box row
     volatile int *abort = &sm.abort;
-    BlockWalker w;
+    BlockWalker<> w;
     w.init(meta, p);
     for (int g = 0; w.live; w.advance(p), ++g) {
         const int s = g % kStages;
@@ -282,13 +349,13 @@ __device__ void convert_warp(Smem &sm, const DecodeParams &p, const int32_t *met
 // accumulator; the next block's Gemm1 may start as soon as the softmax warps have read S.
 // fp8 cache: the 16 latent MMAs are fp16 x fp16 (Q converted on load, K from the converted
 // buffer), the 2 rotary MMAs stay bf16 x bf16 from the raw stage; both accumulate in fp32.
-template <bool F8>
+template <bool F8, bool SP>
 __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
     constexpr uint32_t id1 = idesc_bf16_f32(128, 64, 0);  // S = Q K^T: K-major B
     constexpr uint32_t id1_lat = F8 ? idesc_f16_f32(128, 64, 0) : id1;
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
-    BlockWalker w;
+    BlockWalker<SP> w;
     w.init(meta, p);
     for (int g = 0; w.live; w.advance(p), ++g) {
         if (w.first() && !warp_wait(&sm.q_full, w.piece_k & 1, abort, lane)) break;
@@ -296,6 +363,7 @@ __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
         if (!warp_wait(F8 ? &sm.conv_full[s] : &sm.kv_full[s], (g / kStages) & 1, abort, lane)) break;
         if (g > 0 && !warp_wait(&sm.s_free, (g - 1) & 1, abort, lane)) break;
         if (lane == 0) {
+            if constexpr (SP) fence_proxy_async_smem();  // the gathered stage (generic-proxy copies) to the tensor core
             tc_fence_after();
             // descriptors: one base each, then constant offsets (address field is in 16-byte units)
             const uint64_t kd = smem_desc(smem_addr(sm.stage[s]), 16, 1024, 2);
@@ -316,13 +384,13 @@ __device__ void gemm1_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
 
 // Gemm2 of every block, O (+)= (P_hi + P_lo) V, once the softmax warps have written P.
 // fp8 cache: O (+)= P V with P and V in fp16, 4 MMAs.
-template <bool F8>
+template <bool F8, bool SP>
 __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem) {
     constexpr uint32_t id2 = F8 ? idesc_f16_f32(128, 256, 1) : idesc_bf16_f32(128, 256, 1);  // MN-major B
     constexpr int kTerms = F8 ? 1 : 2;
     const int lane = threadIdx.x & 31;
     volatile int *abort = &sm.abort;
-    BlockWalker w;
+    BlockWalker<SP> w;
     w.init(meta, p);
     for (int g = 0; w.live; w.advance(p), ++g) {
         if (!warp_wait(&sm.p_full, g & 1, abort, lane)) break;
@@ -330,8 +398,10 @@ __device__ void gemm2_warp(Smem &sm, const DecodeParams &p, const int32_t *meta,
         const int s = g % kStages;
         // P of block g exists, so Gemm1 of block g has completed and its tile may be edited (the fp8
         // path's converter has already zeroed the tail rows)
-        if (!F8 && w.tail()) zero_tail_rows(sm.stage[s], w.pc.n - w.blk * kBlk, lane);
+        // (sparse mode: entries that are no key were copied as zeros)
+        if (!F8 && !SP && w.tail()) zero_tail_rows(sm.stage[s], w.pc.n - w.blk * kBlk, lane);
         if (lane == 0) {
+            if constexpr (SP) fence_proxy_async_smem();
             tc_fence_after();
             const uint64_t vd = smem_desc(smem_addr(sm.stage[s]), 4 * 2048, 1024, 2);
             const bool first = w.first();
@@ -434,6 +504,11 @@ __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &
 
 // Own partial scores of block g for this thread's 32 tokens (raw, unscaled); keys at or past `vis`
 // become -inf. The accumulators are released as soon as the scores are in registers.
+// Sparse mode: keys are the stage's validity mask bits instead (then `nvalid` holds this thread's
+// 32 bits of it); the mask was stored before the producer's arrival on kv_full, which this thread
+// waits for itself (it completed before Gemm1, and the stage is not refilled before Gemm2 of this
+// block, which needs this thread's P).
+template <bool SP>
 __device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int key0, int vis, float (&s)[kTokPer],
                                          int &nvalid) {
     if (!mbar_wait(&sm.s_full, g & 1, &sm.abort)) return false;
@@ -448,11 +523,20 @@ __device__ __forceinline__ bool load_raw(Smem &sm, const SoftCtx &c, int g, int 
     tc_fence_before();
     __syncwarp();
     if (c.lane == 0) mbar_arrive(&sm.s_free);
-    const int k0 = key0 + kTokPer * c.th;
-    nvalid = min(max(vis - k0, 0), kTokPer);  // the valid tokens are a prefix of the thread's 32
-    if (k0 + kTokPer > vis) {  // the sequence ends (or the causal limit falls) inside these tokens
+    if constexpr (SP) {
+        const int st = g % kStages;
+        if (!mbar_wait(&sm.kv_full[st], (g / kStages) & 1, &sm.abort)) return false;
+        const uint32_t m = (uint32_t)(sm.vmask[st] >> (kTokPer * c.th));
+        nvalid = (int)m;
 #pragma unroll
-        for (int j = 0; j < kTokPer; ++j) s[j] = k0 + j < vis ? s[j] : -INFINITY;
+        for (int j = 0; j < kTokPer; ++j) s[j] = (m >> j) & 1u ? s[j] : -INFINITY;
+    } else {
+        const int k0 = key0 + kTokPer * c.th;
+        nvalid = min(max(vis - k0, 0), kTokPer);  // the valid tokens are a prefix of the thread's 32
+        if (k0 + kTokPer > vis) {  // the sequence ends (or the causal limit falls) inside these tokens
+#pragma unroll
+            for (int j = 0; j < kTokPer; ++j) s[j] = k0 + j < vis ? s[j] : -INFINITY;
+        }
     }
     return true;
 }
@@ -506,10 +590,10 @@ __device__ __forceinline__ float exps_in_place(float (&s)[kTokPer], float sl2) {
 // 32 factors (`mn`, per token parity) shows whether any is below 2^-14 (valid tokens of rows whose
 // partial maxima overstate the true maximum by ~58 octaves or more; masked tokens carry R' = 0).
 // Only then is the bound summed (the warp votes, so that it branches once).
-// The bound above for tokens 8 c4 .. 8 c4 + 7 of this thread (those below `nv` are valid), in units
-// of l. `w4`: their peer factors (fp16 pairs); `pk`/`pl`: P as stored for Gemm2 (bf16 hi/lo pairs;
+// The bound above for tokens 8 c4 .. 8 c4 + 7 of this thread (those below `nv` are valid; sparse
+// mode: those whose bit is set in `nv`), in units of l. `w4`: their peer factors (fp16 pairs); `pk`/`pl`: P as stored for Gemm2 (bf16 hi/lo pairs;
 // fp8 cache: fp16 pairs in `pk`).
-template <bool F8>
+template <bool F8, bool SP>
 __device__ __forceinline__ float range_excess8(const uint32_t (&w4)[4], int c4, const uint32_t (&pk)[kTokPer / 2],
                                                const uint32_t (&pl)[kTokPer / 2], int nv, float fh) {
     float sq = 0.f;
@@ -517,7 +601,8 @@ __device__ __forceinline__ float range_excess8(const uint32_t (&w4)[4], int c4, 
     for (int k = 0; k < 8; ++k) {
         const int j = 8 * c4 + k, sh = 16 * (k & 1);
         const uint32_t hb = (w4[k >> 1] >> sh) & 0xffffu;
-        if (hb >= 0x400u || j >= nv) continue;  // normal, or a masked token
+        const bool key = SP ? (((uint32_t)nv >> j) & 1u) != 0u : j < nv;
+        if (hb >= 0x400u || !key) continue;  // normal, or a masked token
         const float rp = __half2float(__ushort_as_half((unsigned short)hb));
         float pj;
         if constexpr (F8) {
@@ -531,7 +616,7 @@ __device__ __forceinline__ float range_excess8(const uint32_t (&w4)[4], int c4, 
     return sq;
 }
 
-template <bool F8>
+template <bool F8, bool SP>
 __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t tmem, uint32_t half,
                              int group) {
     SoftCtx c;
@@ -561,18 +646,18 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     const int bar_id = 1 + wq;  // the two warps of these 32 rows
 
     // w walks one block ahead of the block being finished; of that block only a few facts are kept
-    BlockWalker w;
+    BlockWalker<SP> w;
     w.init(meta, p);
     if (!w.live) return;
     load_q<F8>(sm, c, w.pc);
     int vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
     float e_own[kTokPer], m_own;
     int nv_own;  // valid tokens of the block being finished, among this thread's 32
-    if (!load_raw(sm, c, 0, w.blk * kBlk, vis, e_own, nv_own)) return;
+    if (!load_raw<SP>(sm, c, 0, w.blk * kBlk, vis, e_own, nv_own)) return;
     m_own = exps_in_place(e_own, sl2);
     send_factors(c, 0, e_own, m_own);
     if (w.last()) {  // the next piece's Q may replace this one once its last Gemm1 is done
-        Cursor tmp = w.cur;
+        Cursor<SP> tmp = w.cur;
         Piece nx;
         if (tmp.next(p, nx)) load_q<F8>(sm, c, nx);
     }
@@ -589,9 +674,9 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         int nv_nx = 0;
         if (nx_live) {
             if (w.first()) vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
-            if (!load_raw(sm, c, g + 1, w.blk * kBlk, vis, snx, nv_nx)) return;
+            if (!load_raw<SP>(sm, c, g + 1, w.blk * kBlk, vis, snx, nv_nx)) return;
             if (w.last()) {
-                Cursor tmp = w.cur;
+                Cursor<SP> tmp = w.cur;
                 Piece nx;
                 if (tmp.next(p, nx)) load_q<F8>(sm, c, nx);
             }
@@ -747,7 +832,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const uint4 v = xe[((slot * kTq + c.th) * 4 + c4) * 128 + c.i];
                     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                    sq += range_excess8<F8>(w4, c4, pk, pl, nv_own, fh);
+                    sq += range_excess8<F8, SP>(w4, c4, pk, pl, nv_own, fh);
                 }
                 lost += sq;
             }
@@ -790,7 +875,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const uint32_t w4[4] = {ep[4 * c4], ep[4 * c4 + 1], ep[4 * c4 + 2], ep[4 * c4 + 3]};
-                    sq += range_excess8<F8>(w4, c4, pk, pl, nv_own, fh);
+                    sq += range_excess8<F8, SP>(w4, c4, pk, pl, nv_own, fh);
                 }
                 lost += sq;
             }
@@ -856,7 +941,8 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                 if (c.row_ok && half == 0 && c.th == 0) {
                     const float lse = empty ? -INFINITY : (m_ref + log2f(l_row)) * 0.69314718055994530942f;
                     if (whole)
-                        p.lse[((size_t)a_seq * p.h_q + h_idx) * p.s_q + t_q] = lse;
+                        p.lse[SP ? ((size_t)(a_seq / p.sp_sq) * p.h_q + h_idx) * p.sp_sq + a_seq % p.sp_sq
+                                 : ((size_t)a_seq * p.h_q + h_idx) * p.s_q + t_q] = lse;
                     else
                         p.lse_part[(size_t)a_slot * p.rows + c.r] = lse;
                 }
@@ -874,7 +960,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     }
 }
 
-template <bool F8>
+template <bool F8, bool SP>
 __global__ void __launch_bounds__(num_threads<F8>(), 1)
 decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_rope,
                     const DecodeParams p, const int groups) {
@@ -889,7 +975,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);  // whole (converged) warp
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_full[s], SP ? 33 : 1);  // sparse: 32 lanes' copies + the mask
             mbar_init(&sm.kv_empty[s], 1);
             mbar_init(&sm.conv_full[s], kConvWarps);
         }
@@ -906,7 +992,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
         sm.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (!SP && warp == 0 && lane == 0) {
         prefetch_tensormap(&map_lat);
         prefetch_tensormap(&map_rope);
     }
@@ -922,19 +1008,22 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     } else if (warp < 4) {
         setmaxnreg_dec<F8 ? kRegsSmall : kRegsControl>();
         if (warp == 0) {
-            if (lane == 0) producer<F8>(sm, p, &map_lat, &map_rope, meta, half);
+            if constexpr (SP)
+                gather_producer(sm, p, meta, half);
+            else if (lane == 0)
+                producer<F8>(sm, p, &map_lat, &map_rope, meta, half);
         } else {
             if (warp == 3) {
-                gemm2_warp<F8>(sm, p, meta, tmem);
+                gemm2_warp<F8, SP>(sm, p, meta, tmem);
                 drain_mmas(sm);
             } else if (warp == 1) {
-                gemm1_warp<F8>(sm, p, meta, tmem);
+                gemm1_warp<F8, SP>(sm, p, meta, tmem);
                 drain_mmas(sm);
             }
         }
     } else {
         setmaxnreg_inc<kRegsSoftmax>();
-        softmax_role<F8>(sm, p, meta, tmem, half, group);
+        softmax_role<F8, SP>(sm, p, meta, tmem, half, group);
     }
     __syncwarp();
     tc_fence_before();
@@ -951,11 +1040,15 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
 
 size_t decode_sm100_smem_bytes() { return sizeof(dec::Smem) + 1024; }
 
+// sparse (p.indices set) runs the bf16-cache kernel with the gather producer; the maps are then unused.
 cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_lat, const CUtensorMap &map_rope,
                                 bool fp8, cudaStream_t stream) {
     const int groups = (p.rows + 127) / 128;
     const size_t smem = decode_sm100_smem_bytes();
-    auto kernel = fp8 ? dec::decode_sm100_kernel<true> : dec::decode_sm100_kernel<false>;
+    const bool sparse = p.indices != nullptr;
+    if (fp8 && sparse) return cudaErrorInvalidValue;
+    auto kernel = fp8 ? dec::decode_sm100_kernel<true, false>
+                      : (sparse ? dec::decode_sm100_kernel<false, true> : dec::decode_sm100_kernel<false, false>);
     const int threads = fp8 ? dec::num_threads<true>() : dec::num_threads<false>();
     // setmaxnreg redistributes the registers the block was launched with: the warpgroups' shares must
     // fit in what the compiler gave the kernel, or the raising warps would wait forever

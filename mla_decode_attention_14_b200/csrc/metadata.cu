@@ -10,6 +10,9 @@
 // T = max(1, ceil(U/P)) and the block at unit u belongs to part floor(u/T). So every part
 // is a contiguous run of (sequence, block) pairs and its work is at most T + C units.
 //
+// Sparse mode gives every work unit the same length (its index list); `seqlens` is then null
+// and `uniform_n` that length.
+//
 // This kernel derives each part's bounds in closed form from the prefix sums of the
 // per-sequence costs: one CTA, a chunked block-wide scan over the sequences, and each
 // sequence writes the begin/end fields of the parts its blocks touch (every field is
@@ -49,7 +52,7 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T *warp_sums, T *total) {
 }
 
 __global__ void __launch_bounds__(kMetaThreads)
-metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int num_parts, int C,
+metadata_kernel(const int32_t *__restrict__ seqlens, int uniform_n, int batch, int num_parts, int C,
                 int32_t *__restrict__ tile_meta, int32_t *__restrict__ num_splits) {
     __shared__ int64_t warp_sums64[32];
     __shared__ int32_t warp_sums32[32];
@@ -64,7 +67,7 @@ metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int num_parts, i
     // pass 1: total units U
     int64_t local = 0;
     for (int i = threadIdx.x; i < batch; i += blockDim.x) {
-        int w = num_blocks_of(seqlens[i]);
+        int w = num_blocks_of(seqlens ? seqlens[i] : uniform_n);
         if (w > 0) local += (int64_t)C + w;
     }
 #pragma unroll
@@ -83,7 +86,7 @@ metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int num_parts, i
     int32_t carry_splits = 0;
     for (int base = 0; base < batch; base += blockDim.x) {
         const int i = base + threadIdx.x;
-        const int w = i < batch ? num_blocks_of(seqlens[i]) : 0;
+        const int w = i < batch ? num_blocks_of(seqlens ? seqlens[i] : uniform_n) : 0;
         const int64_t cost = w > 0 ? (int64_t)C + w : 0;
         int64_t chunk_units;
         const int64_t pre = carry_units + block_exclusive_scan<int64_t>(cost, warp_sums64, &chunk_units);
@@ -116,9 +119,9 @@ metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int num_parts, i
     }
 }
 
-cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, int fixed_cost,
+cudaError_t launch_metadata(const int32_t *seqlens, int uniform_n, int batch, int num_parts, int fixed_cost,
                             int32_t *tile_meta, int32_t *num_splits, cudaStream_t stream) {
-    metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, batch, num_parts, fixed_cost,
+    metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, uniform_n, batch, num_parts, fixed_cost,
                                                     tile_meta, num_splits);
     return cudaGetLastError();
 }

@@ -17,6 +17,8 @@ struct Piece {
 };
 
 // Walks the non-empty pieces of one part (all roles walk the same list independently).
+// SP: sparse mode, where every work unit has topk keys (its index list).
+template <bool SP = false>
 struct Cursor {
     int seq, begin_seq, begin_blk, end_seq, end_blk, first_piece;
     __device__ void init(const int32_t *meta, int batch) {
@@ -31,7 +33,7 @@ struct Cursor {
     __device__ bool next(const DecodeParams &p, Piece &pc) {
         while (seq <= end_seq) {
             const int s = seq++;
-            const int n = max(p.seqlens[s], 0);
+            const int n = SP ? p.topk : max(p.seqlens[s], 0);
             const int w = num_blocks_of(n);
             const int lo = s == begin_seq ? max(begin_blk, 0) : 0;
             const int hi = s == end_seq ? min(end_blk, w) : w;

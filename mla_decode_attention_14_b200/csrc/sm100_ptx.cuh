@@ -369,3 +369,20 @@ __device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
 }
 }  // namespace sm100
 }  // namespace mla
+
+namespace mla {
+namespace sm100 {
+// 16-byte asynchronous global -> shared copy (L2 only); src_bytes 0 writes 16 zero bytes and reads
+// nothing.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrive on `bar` once every asynchronous copy this thread has issued has completed; the arrival is
+// one of the barrier's expected arrivals (noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+// Wait until every asynchronous copy this thread has issued has completed.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+}  // namespace sm100
+}  // namespace mla

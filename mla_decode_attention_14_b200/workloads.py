@@ -206,6 +206,33 @@ def make_inputs_fp8(wl: Workload, seed: int = 0, tail: str = "nan", spare_blocks
             "scale": wl.scale, "causal": wl.causal, "num_blocks": nblk}
 
 
+def sparse_indices(seqlens, s_q: int, topk: int, seed: int = 0, order: str = "sorted") -> np.ndarray:
+    """Index lists for sparse decode: int32 [b, s_q, topk] positions within each sequence.
+
+    Each (sequence, query token) draws ``min(topk, n)`` distinct positions of its sequence
+    uniformly; lists longer than the sequence are padded with -1 (no key). ``order``: "sorted"
+    (ascending positions) or "shuffled".
+    """
+    sl = np.asarray(seqlens, dtype=np.int64)
+    rng = np.random.default_rng([seed, 4])
+    out = np.full((sl.shape[0], s_q, topk), -1, dtype=np.int32)
+    for b, n in enumerate(sl):
+        n = max(int(n), 0)
+        k = min(topk, n)
+        for t in range(s_q):
+            if k == 0:
+                continue
+            pos = rng.choice(n, size=k, replace=False) if k < n else np.arange(n)
+            if order == "sorted":
+                pos = np.sort(pos)
+            elif order == "shuffled":
+                pos = rng.permutation(pos)
+            else:
+                raise ValueError(order)
+            out[b, t, :k] = pos
+    return out
+
+
 def algorithmic_counts(wl: Workload, kv: str = "bf16"):
     """Algorithmic bytes and flops of one decode of ``wl``.
 
