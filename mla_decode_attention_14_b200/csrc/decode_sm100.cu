@@ -73,15 +73,18 @@ constexpr int kStages = 5;
 constexpr int kSoftWarps = 8;                     // two per SM sub-partition
 // bf16 cache: warpgroup 0 = TMA producer, Gemm1 issuer, (idle), Gemm2 issuer; softmax from warp 4.
 // fp8 cache: warpgroup 1 = four converter warps (one per SM sub-partition); softmax from warp 8.
+// sparse mode (bf16 cache): warpgroup 1 = four gather warps; softmax from warp 8.
 constexpr int kConvWarps = 4;
-template <bool F8> constexpr int first_soft_warp() { return F8 ? 4 + kConvWarps : 4; }
-template <bool F8> constexpr int num_threads() { return 32 * (first_soft_warp<F8>() + kSoftWarps); }  // 384 / 512
+template <bool F8, bool SP = false> constexpr int first_soft_warp() { return (F8 || SP) ? 4 + kConvWarps : 4; }
+template <bool F8, bool SP = false> constexpr int num_threads() {
+    return 32 * (first_soft_warp<F8, SP>() + kSoftWarps);  // 384 / 512
+}
 constexpr int kTq = 2;                            // token halves per block
 constexpr int kTokPer = kBlk / kTq;               // 32 tokens per softmax thread
 // Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 = 64,512); warpgroup 0
 // drops to 96 and the two softmax warpgroups rise to 200: 128 x 96 + 256 x 200 = 63,488 <= 64,512.
-// fp8: 512 x 128 = 65,536 at launch; the control and converter warpgroups drop to 56:
-// 2 x 128 x 56 + 256 x 200 = 65,536.
+// fp8 and sparse: 512 x 128 = 65,536 at launch; the control and converter (gather) warpgroups drop
+// to 56: 2 x 128 x 56 + 256 x 200 = 65,536.
 constexpr uint32_t kRegsControl = 96, kRegsSoftmax = 200, kRegsSmall = 56;
 constexpr int kBoxBytes = kBlk * 128;                      // 64 tokens x 64 bf16 (128-byte swizzle)
 constexpr int kRopeBoxBytes = kBlk * 64;                   // 64 tokens x 32 bf16 (64-byte swizzle)
@@ -201,51 +204,77 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// ---------------------------------------------------------------- sparse mode: gather producer (1 warp)
-// Block k of work unit u holds the keys listed at indices[u, 64k .. 64k+64). Lane l resolves
-// entries l and l + 32: a position inside [0, seqlens[b]) is a key, read from cache row
-// block_table[b, pos / 64] * 64 + pos % 64; anything else (or a list shorter than the block) is no
-// key, copied as zeros. Then, token by token, the 32 lanes copy this CTA's 512-byte latent half of
-// the row, one 16-byte chunk each (one coalesced 512-byte read), and lanes 0-3 its 64-byte rotary
-// half, with 16-byte asynchronous copies into the positions the stage's 128-byte (latent) and
-// 64-byte (rotary) swizzles give them -- the layout the MMA descriptors read, which a TMA box cannot
-// produce for single rows. The stage's validity mask is stored before lane 0's arrival on kv_full;
-// each lane's copies complete on kv_full too (33 arrivals per fill).
-__device__ void gather_producer(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t half) {
+// ---------------------------------------------------------------- sparse mode: gather producers (4 warps)
+// Block k of work unit u holds the keys listed at indices[u, 64k .. 64k+64). Gather warp h (warps
+// 4-7) takes the block's tokens [16h, 16h + 16); its lane l < 16 resolves entry 16h + l: a position
+// inside [0, seqlens[b]) is a key, read from cache row block_table[b, pos / 64] * 64 + pos % 64;
+// anything else (or a list shorter than the block) is no key, copied as zeros. Then, token by
+// token, the warp's 32 lanes copy this CTA's 512-byte latent half of the row, one 16-byte chunk
+// each (one coalesced 512-byte read), and lanes 0-3 its 64-byte rotary half, with 16-byte
+// asynchronous copies into the positions the stage's 128-byte (latent) and 64-byte (rotary)
+// swizzles give them -- the layout the MMA descriptors read, which a TMA box cannot produce for
+// single rows. Each warp stores its quarter of the stage's validity mask before its lane 0 arrives on
+// kv_full, and each lane's copies complete on kv_full too (4 x 33 arrivals per fill).
+// A warp keeps only ~9 KB of such copies in flight (measured: ~6k cycles to issue one block's
+// 36 KB from one warp, ~3.5k from two), so the copies are split over a warpgroup. Resolving an entry takes two
+// dependent loads (list, then block table), so the walk is pipelined: while block g is copied, the
+// block-table entry of block g+1 and the list entry (and sequence length) of block g+2 are in flight.
+constexpr int kGatherWarps = 4;
+constexpr int kGatherTok = kBlk / kGatherWarps;  // 16 tokens of each block per gather warp
+constexpr uint32_t kSparseFullArrivals = kGatherWarps * 33;
+
+struct GatherAhead {  // this lane's list entry of one block, loaded ahead
+    int pos, n, b;
+};
+
+__device__ __forceinline__ void gather_load_list(const DecodeParams &p, const BlockWalker<true> &w, int e_off,
+                                                 GatherAhead &a) {
+    a.b = w.live ? w.pc.seq / p.sp_sq : 0;
+    a.n = w.live ? max(__ldg(&p.seqlens[a.b]), 0) : 0;
+    const int e = w.blk * kBlk + e_off;  // e_off < 0: this lane has no entry
+    a.pos = w.live && e_off >= 0 && e < p.topk ? __ldg(&p.indices[(size_t)w.pc.seq * p.topk + e]) : -1;
+}
+
+// the cache row (physical block * 64 + slot) of the entry, or -1
+__device__ __forceinline__ int gather_resolve(const DecodeParams &p, const GatherAhead &a, bool &bad_entry) {
+    const int pos = a.pos;
+    if (pos < 0 || pos >= a.n) return -1;
+    const int blk = pos / kBlk;
+    const int phys = blk < p.bt_stride ? __ldg(&p.block_table[(size_t)a.b * p.bt_stride + blk]) : -1;
+    if (phys >= 0 && (int64_t)phys < p.num_blocks) return phys * kBlk + pos % kBlk;
+    bad_entry = true;  // reported; the entry is treated as no key
+    return -1;
+}
+
+__device__ void gather_producer(Smem &sm, const DecodeParams &p, const int32_t *meta, uint32_t half, int gw) {
     const int lane = threadIdx.x & 31;
+    const int t0 = kGatherTok * gw;  // this warp's tokens of each block
+    const int e_off = lane < kGatherTok ? t0 + lane : -1;  // lanes past the warp's tokens resolve nothing
     volatile int *abort = &sm.abort;
     const char *kv = reinterpret_cast<const char *>(p.kv);
-    BlockWalker<true> w;
-    w.init(meta, p);
-    int gidx = 0;
     bool bad_entry = false;
+    // w: the block being copied; w2: two blocks ahead (its list entries are loaded)
+    BlockWalker<true> w, w2;
+    w.init(meta, p);
+    w2 = w;
+    GatherAhead a1, a2;  // list entries of blocks g+1 and g+2
+    gather_load_list(p, w, e_off, a1);
+    int row = gather_resolve(p, a1, bad_entry);  // block g
+    if (w2.live) w2.advance(p);
+    gather_load_list(p, w2, e_off, a1);
+    if (w2.live) w2.advance(p);
+    int gidx = 0;
     for (; w.live; w.advance(p), ++gidx) {
+        gather_load_list(p, w2, e_off, a2);  // block g+2
+        if (w2.live) w2.advance(p);
         const int s = gidx % kStages, fill = gidx / kStages;
         if (fill > 0 && !warp_wait(&sm.kv_empty[s], (fill - 1) & 1, abort, lane)) break;
-        const int b = w.pc.seq / p.sp_sq;
-        const int n = max(__ldg(&p.seqlens[b]), 0);
-        const int32_t *list = p.indices + (size_t)w.pc.seq * p.topk;
-        int row[2];  // cache row (physical block * 64 + slot) of entries lane and lane + 32, or -1
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = w.blk * kBlk + 32 * u + lane;
-            const int pos = e < p.topk ? __ldg(&list[e]) : -1;
-            row[u] = -1;
-            if (pos >= 0 && pos < n) {
-                const int blk = pos / kBlk;
-                const int phys = blk < p.bt_stride ? __ldg(&p.block_table[(size_t)b * p.bt_stride + blk]) : -1;
-                if (phys >= 0 && (int64_t)phys < p.num_blocks)
-                    row[u] = phys * kBlk + pos % kBlk;
-                else
-                    bad_entry = true;  // reported; the entry is treated as no key
-            }
-        }
-        const uint64_t mask = (uint64_t)__ballot_sync(0xffffffffu, row[0] >= 0) |
-                              ((uint64_t)__ballot_sync(0xffffffffu, row[1] >= 0) << 32);
+        const uint32_t mask = __ballot_sync(0xffffffffu, row >= 0) & ((1u << kGatherTok) - 1);
         const uint32_t dst = smem_addr(sm.stage[s]);
 #pragma unroll 4
-        for (int t = 0; t < kBlk; ++t) {
-            const int r = __shfl_sync(0xffffffffu, t < 32 ? row[0] : row[1], t & 31);
+        for (int k = 0; k < kGatherTok; ++k) {
+            const int t = t0 + k;
+            const int r = __shfl_sync(0xffffffffu, row, k);
             const uint32_t bytes = r >= 0 ? 16u : 0u;  // 0: the chunk is zero-filled, nothing is read
             const char *src = kv + (size_t)(r >= 0 ? r : 0) * (kDqk * 2);
             // latent chunk `lane` of this half: dims 256 half + 8 lane, box lane / 8, chunk lane % 8
@@ -256,10 +285,12 @@ __device__ void gather_producer(Smem &sm, const DecodeParams &p, const int32_t *
                             src + (512 + 32 * half + 8 * lane) * 2, bytes);
         }
         if (lane == 0) {
-            sm.vmask[s] = mask;
+            reinterpret_cast<uint16_t *>(&sm.vmask[s])[gw] = (uint16_t)mask;  // bits 16 gw .. 16 gw + 15
             mbar_arrive(&sm.kv_full[s]);
         }
         cp_async_mbar_arrive_noinc(&sm.kv_full[s]);
+        row = gather_resolve(p, a1, bad_entry);  // block g+1
+        a1 = a2;
     }
     if (bad_entry) raise_error(kErrBounds);
     cp_async_wait_all();  // every copy lands before the CTA may exit
@@ -625,7 +656,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     c.half = half;
     const int warp = threadIdx.x >> 5;
     const int wq = warp & 3;
-    c.th = (warp - first_soft_warp<F8>()) >> 2;
+    c.th = (warp - first_soft_warp<F8, SP>()) >> 2;
     c.lane = threadIdx.x & 31;
     c.i = wq * 32 + c.lane;  // row within the group == TMEM lane
     c.lane_off = (uint32_t)(wq * 32) << 16;
@@ -686,7 +717,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         }
         // peer factors of block g (slot g % 2)
         const int slot = g & 1;
-        if (threadIdx.x == 32 * first_soft_warp<F8>()) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
+        if (threadIdx.x == 32 * first_soft_warp<F8, SP>()) mbar_arrive_expect_tx(&sm.xfull[slot], xbytes);
         if (!mbar_wait_cluster(&sm.xfull[slot], (g >> 1) & 1, abort)) return;
         const float m_peer = c.warp_ok ? xo[(slot * kTq + c.th) * 128 + c.i] : -INFINITY;
         const float mbu_half = m_own + m_peer;
@@ -961,7 +992,7 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
 }
 
 template <bool F8, bool SP>
-__global__ void __launch_bounds__(num_threads<F8>(), 1)
+__global__ void __launch_bounds__(num_threads<F8, SP>(), 1)
 decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_rope,
                     const DecodeParams p, const int groups) {
     extern __shared__ uint8_t smem_raw[];
@@ -975,7 +1006,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);  // whole (converged) warp
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.kv_full[s], SP ? 33 : 1);  // sparse: 32 lanes' copies + the mask
+            mbar_init(&sm.kv_full[s], SP ? kSparseFullArrivals : 1);  // sparse: the gather warps' copies + masks
             mbar_init(&sm.kv_empty[s], 1);
             mbar_init(&sm.conv_full[s], kConvWarps);
         }
@@ -1002,16 +1033,18 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_co
     cluster_sync();  // the peer's barriers exist before any exchange targets them
     const uint32_t tmem = sm.tmem_base;
 
-    if (F8 && warp >= 4 && warp < first_soft_warp<F8>()) {
+    if ((F8 || SP) && warp >= 4 && warp < first_soft_warp<F8, SP>()) {
         setmaxnreg_dec<kRegsSmall>();
-        convert_warp(sm, p, meta);
+        if constexpr (SP)
+            gather_producer(sm, p, meta, half, warp - 4);
+        else
+            convert_warp(sm, p, meta);
     } else if (warp < 4) {
-        setmaxnreg_dec<F8 ? kRegsSmall : kRegsControl>();
-        if (warp == 0) {
-            if constexpr (SP)
-                gather_producer(sm, p, meta, half);
-            else if (lane == 0)
-                producer<F8>(sm, p, &map_lat, &map_rope, meta, half);
+        setmaxnreg_dec<(F8 || SP) ? kRegsSmall : kRegsControl>();
+        if (SP && warp == 0) {
+            // sparse: warpgroup 1 gathers; warp 0 has nothing to do
+        } else if (warp == 0) {
+            if (lane == 0) producer<F8>(sm, p, &map_lat, &map_rope, meta, half);
         } else {
             if (warp == 3) {
                 gemm2_warp<F8, SP>(sm, p, meta, tmem);
@@ -1049,11 +1082,11 @@ cudaError_t launch_decode_sm100(const DecodeParams &p, const CUtensorMap &map_la
     if (fp8 && sparse) return cudaErrorInvalidValue;
     auto kernel = fp8 ? dec::decode_sm100_kernel<true, false>
                       : (sparse ? dec::decode_sm100_kernel<false, true> : dec::decode_sm100_kernel<false, false>);
-    const int threads = fp8 ? dec::num_threads<true>() : dec::num_threads<false>();
+    const int threads = fp8 ? dec::num_threads<true>() : (sparse ? dec::num_threads<false, true>() : dec::num_threads<false>());
     // setmaxnreg redistributes the registers the block was launched with: the warpgroups' shares must
     // fit in what the compiler gave the kernel, or the raising warps would wait forever
-    const int need = fp8 ? 2 * 128 * (int)dec::kRegsSmall + 256 * (int)dec::kRegsSoftmax
-                         : 128 * (int)dec::kRegsControl + 256 * (int)dec::kRegsSoftmax;
+    const int need = (fp8 || sparse) ? 2 * 128 * (int)dec::kRegsSmall + 256 * (int)dec::kRegsSoftmax
+                                     : 128 * (int)dec::kRegsControl + 256 * (int)dec::kRegsSoftmax;
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
     if (e != cudaSuccess) return e;

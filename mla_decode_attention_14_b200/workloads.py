@@ -233,6 +233,18 @@ def sparse_indices(seqlens, s_q: int, topk: int, seed: int = 0, order: str = "so
     return out
 
 
+def sparse_counts(wl: Workload, indices: np.ndarray):
+    """Algorithmic bytes and flops of one sparse decode: 1152 bytes per listed key that is a key
+    (a position inside its sequence) plus 1152 per query row; 2 * (576 + 512) flops per (key, row)."""
+    n = np.maximum(wl.seqlens.astype(np.int64), 0)
+    ix = np.asarray(indices)
+    keys = int(((ix >= 0) & (ix < n[:, None, None])).sum())
+    kv_bytes = keys * D_QK * 2
+    q_bytes = wl.batch * wl.rows * D_QK * 2
+    return {"kv_bytes": kv_bytes, "q_bytes": q_bytes, "bytes": kv_bytes + q_bytes,
+            "flops": keys * wl.h_q * 2 * (D_QK + D_V)}
+
+
 def algorithmic_counts(wl: Workload, kv: str = "bf16"):
     """Algorithmic bytes and flops of one decode of ``wl``.
 
