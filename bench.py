@@ -42,8 +42,12 @@ from mla_decode_attention_14_b200 import workloads as W  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+SPEC_HBM_GBS = 8000.0         # B200 HBM3e, nominal (7.7 TB/s in HGX systems)
+SPEC_BF16_TFLOPS = 2250.0     # B200 dense bf16/fp16 tensor peak, nominal
+TARGET_HBM_FRAC = 0.80        # the split kernel's goal on the v3 workload
 METRIC = "MLA decode effective TB/s and TFLOPS vs B200 roofline (bf16 paged KV)"
 METRIC_FP8 = "MLA decode effective TB/s and TFLOPS vs B200 roofline (fp8 paged KV)"
+METRIC_SPARSE = "MLA sparse decode effective TB/s and TFLOPS vs B200 roofline (bf16 paged KV, top-k lists)"
 PROFILE_TRAFFIC = {"bf16": os.path.join(ROOT, "profiles", "decode_split_v3_traffic.txt"),
                    "fp8": os.path.join(ROOT, "profiles", "decode_split_fp8_v3_traffic.txt")}
 L2_BYTES = 126 << 20
@@ -90,7 +94,7 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
-SPLIT_KERNEL_SOURCES = ("common.cuh", "decode_sm100.cu", "sm100_ptx.cuh")  # the split kernel's device code
+SPLIT_KERNEL_SOURCES = ("common.cuh", "decode_sm100.cu", "sm100_ptx.cuh", "schedule.cuh")  # the split kernel's device code
 
 
 def kernel_source_hash() -> str:
@@ -325,6 +329,113 @@ def neighbour_steps(mla, wl, dev, stream, iters=50):
     return res
 
 
+# --------------------------------------------------------------------------- every workload
+CONFIG_SET = [("tiny", "bf16", None), ("v2lite", "bf16", None), ("multitoken", "bf16", None),
+              ("skewed", "bf16", None), ("v2lite", "fp8", None), ("v3", "fp8", None),
+              ("multitoken", "fp8", None), ("skewed", "fp8", None), ("v3", "bf16", 2048)]
+
+
+def roofline_fracs(nbytes: int, flops: int, seconds: float, peaks):
+    hbm, tfl_burst, _, _ = peaks
+    gbs, tf = nbytes / seconds / 1e9, flops / seconds / 1e12
+    ridge = tfl_burst * 1e12 / (hbm * 1e9)
+    return {"bound": "hbm" if flops / nbytes < ridge else "tensor",
+            "hbm_frac": gbs / hbm, "tensor_frac": tf / tfl_burst,
+            "hbm_frac_spec": gbs / SPEC_HBM_GBS, "tensor_frac_spec": tf / SPEC_BF16_TFLOPS}
+
+
+def measure_config(mla, name, kv, topk, dev, stream, peaks, target_s=0.4, warmup=5):
+    """One workload at 1 GPU: whole step (metadata + split + combine) and split kernel, CUDA events."""
+    import torch
+    wl = W.workload(name)
+    fp8 = kv == "fp8"
+    inp = W.make_inputs_fp8(wl, seed=0, tail="normal") if fp8 else W.make_inputs(wl, seed=0, tail="normal")
+    q = torch.from_numpy(inp["q"]).view(torch.bfloat16).to(dev)
+    kvt = (torch.from_numpy(inp["kv8"]) if fp8 else torch.from_numpy(inp["kv"]).view(torch.bfloat16)).to(dev)
+    bt = torch.from_numpy(inp["block_table"]).to(dev)
+    sl = torch.from_numpy(inp["seqlens"]).to(dev)
+    out = torch.empty((wl.batch, wl.s_q, wl.h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.batch, wl.h_q, wl.s_q), dtype=torch.float32, device=dev)
+    if topk:
+        ixh = W.sparse_indices(wl.seqlens, wl.s_q, topk, seed=0)
+        ix = torch.from_numpy(ixh).to(dev)
+        counts = W.sparse_counts(wl, ixh)
+        parts = mla.default_num_parts(wl.h_q, 1, dev)
+        ws = torch.empty((mla.workspace_bytes(wl.batch * wl.s_q, 1, wl.h_q, parts),), dtype=torch.uint8, device=dev)
+
+        def step(ev=None):
+            meta = mla.get_metadata_sparse(wl.batch, wl.s_q, wl.h_q, topk, num_parts=parts)
+            if ev is not None:
+                ev[0].record(stream)
+            mla.decode_sparse(q, kvt, bt, sl, ix, wl.scale, meta, out=out, lse=lse, workspace=ws)
+            if ev is not None:
+                ev[1].record(stream)
+    else:
+        counts = W.algorithmic_counts(wl, kv)
+        parts = mla.default_num_parts(wl.h_q, wl.s_q, dev)
+        ws = torch.empty((mla.workspace_bytes(wl.batch, wl.s_q, wl.h_q, parts),), dtype=torch.uint8, device=dev)
+
+        def dec(meta, phase):
+            if fp8:
+                mla.decode_fp8(q, kvt, bt, sl, wl.scale, inp["kv_scale"], wl.causal, meta, out=out, lse=lse,
+                               workspace=ws, phase=phase)
+            else:
+                mla.decode(q, kvt, bt, sl, wl.scale, wl.causal, meta, out=out, lse=lse, workspace=ws, phase=phase)
+
+        def step(ev=None):
+            meta = mla.get_metadata(sl, wl.h_q, wl.s_q, num_parts=parts)
+            if ev is not None:
+                ev[0].record(stream)
+            dec(meta, "split")
+            if ev is not None:
+                ev[1].record(stream)
+            dec(meta, "combine")
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if mla.check_status() != 0:
+        raise SystemExit("device error status after warm-up of %s/%s" % (name, kv))
+    t0 = time.perf_counter()
+    step()
+    torch.cuda.synchronize()
+    steps = int(min(5000, max(20, target_s / max(time.perf_counter() - t0, 1e-6))))
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev) if counts["bytes"] < 2 * L2_BYTES else None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    whole = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            whole[i][0].record(stream)
+            step(evs[i])
+            whole[i][1].record(stream)
+        torch.cuda.synchronize()
+    if mla.check_status() != 0:
+        raise SystemExit("device error status in the timed region of %s/%s" % (name, kv))
+    step_ms = statistics.mean(a.elapsed_time(b) for a, b in whole)
+    split_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    rec = {"workload": describe(wl, kv) + (", top-%d sparse lists (uniform, sorted)" % topk if topk else ""),
+           "kv": kv, "sparse_topk": topk, "steps": steps, "ms_per_step": step_ms,
+           "value": counts["bytes"] / (step_ms * 1e-3) / 1e12, "unit": "TB/s",
+           "tflops": counts["flops"] / (step_ms * 1e-3) / 1e12,
+           "algorithmic_bytes": counts["bytes"], "algorithmic_flops": counts["flops"],
+           "l2": "flushed between steps (256 MB write, untimed)" if flush is not None else "inputs larger than L2",
+           "clocks": clk.summary()}
+    if topk:  # one call launches both kernels: the step time stands for the kernel
+        rec["split_ms"] = None
+        rec["roofline"] = dict(roofline_fracs(counts["bytes"], counts["flops"], step_ms * 1e-3, peaks),
+                               basis="whole sparse call (split + combine)")
+    else:
+        rec["split_ms"] = split_ms
+        rec["roofline"] = dict(roofline_fracs(counts["bytes"], counts["flops"], split_ms * 1e-3, peaks),
+                               basis="split kernel")
+    del q, kvt, bt, sl, out, lse, ws, flush
+    torch.cuda.empty_cache()
+    return rec
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -339,12 +450,18 @@ def main():
                     help="replays of the step captured in a CUDA graph, reported under 'graph' "
                          "(default: as many as --steps; 0: skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip timing the other workloads (1 GPU only)")
     ap.add_argument("--no-neighbours", action="store_true", help="skip timing the projections and the append")
     ap.add_argument("--max-batch", type=int, default=0,
                     help="keep only the first N sequences (for profiler captures of a smaller slice)")
+    ap.add_argument("--topk", type=int, default=0,
+                    help="sparse decode (bf16 cache): every query token attends to K positions drawn "
+                         "uniformly from its sequence (sorted lists); the headline becomes mla_decode_sparse")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.topk and (args.kv != "bf16" or args.impl != "ours"):
+        ap.error("--topk runs the library's sparse decode over the bf16 cache only")
 
     wl = W.workload(args.workload)
     if args.max_batch and args.max_batch < wl.batch:
@@ -352,6 +469,10 @@ def main():
                       name="%s[:%d]" % (wl.name, args.max_batch))
     counts = W.algorithmic_counts(wl, kv=args.kv)
     fp8 = args.kv == "fp8"
+    topk = args.topk
+    if topk:
+        ixh = W.sparse_indices(wl.seqlens, wl.s_q, topk, seed=0)
+        counts = W.sparse_counts(wl, ixh)
 
     def make_inputs():
         return W.make_inputs_fp8(wl, seed=0, tail="normal") if fp8 else W.make_inputs(wl, seed=0, tail="normal")
@@ -385,9 +506,12 @@ def main():
     kv = (torch.from_numpy(inp["kv8"]) if fp8 else torch.from_numpy(inp["kv"]).view(torch.bfloat16)).to(dev)
     bt = torch.from_numpy(inp["block_table"]).to(dev)
     sl = torch.from_numpy(inp["seqlens"]).to(dev)
-    num_parts = mla.default_num_parts(wl.h_q, wl.s_q, dev)
-    fixed_cost = mla.default_fixed_cost(wl.h_q, wl.s_q)
-    ws = torch.empty((mla.workspace_bytes(wl.batch, wl.s_q, wl.h_q, num_parts),), dtype=torch.uint8, device=dev)
+    num_parts = mla.default_num_parts(wl.h_q, 1 if topk else wl.s_q, dev)
+    fixed_cost = mla.default_fixed_cost(wl.h_q, 1 if topk else wl.s_q)
+    ws_shape = (wl.batch * wl.s_q, 1) if topk else (wl.batch, wl.s_q)
+    ws = torch.empty((mla.workspace_bytes(ws_shape[0], ws_shape[1], wl.h_q, num_parts),), dtype=torch.uint8,
+                     device=dev)
+    ix = torch.from_numpy(ixh).to(dev) if topk else None
     out = torch.empty((wl.batch, wl.s_q, wl.h_q, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((wl.batch, wl.h_q, wl.s_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -399,6 +523,14 @@ def main():
         return mla.decode(q, kv, bt, sl, wl.scale, wl.causal, meta, out=out, lse=lse, workspace=ws, phase=phase)
 
     def step(ev=None):
+        if topk:  # one call launches both kernels: the events bracket the whole call
+            meta = mla.get_metadata_sparse(wl.batch, wl.s_q, wl.h_q, topk, num_parts=num_parts, fixed_cost=fixed_cost)
+            if ev is not None:
+                ev[0].record(stream)
+            mla.decode_sparse(q, kv, bt, sl, ix, wl.scale, meta, out=out, lse=lse, workspace=ws)
+            if ev is not None:
+                ev[1].record(stream)
+            return
         meta = mla.get_metadata(sl, wl.h_q, wl.s_q, num_parts=num_parts, fixed_cost=fixed_cost)
         if ev is not None:
             ev[0].record(stream)
@@ -485,7 +617,7 @@ def main():
 
     # end to end through the host entry point: pinned host inputs in, host outputs out
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not topk:  # the host entry point is the dense decode's
         hd = mla.HostDecoder(wl.batch, wl.s_q, wl.h_q, kv.shape[0], bt.shape[1], device=dev,
                              num_parts=num_parts, fixed_cost=fixed_cost, kv_scale=inp["kv_scale"] if fp8 else None)
         qh = torch.from_numpy(inp["q"]).view(torch.bfloat16).pin_memory()
@@ -511,7 +643,18 @@ def main():
         e2e = {"value": bytes_all / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    neighbours = None if args.no_neighbours or fp8 else neighbour_steps(mla, wl, dev, stream)
+    neighbours = None if args.no_neighbours or fp8 or topk else neighbour_steps(mla, wl, dev, stream)
+
+    # every other workload (and cache format), 1 GPU only: the same step, timed on its own
+    configs = None
+    if world == 1 and not args.no_configs and not topk:
+        peaks = measured_peaks()
+        configs = {}
+        for name, kvk, topk in CONFIG_SET:
+            if name == args.workload and kvk == args.kv and topk is None:
+                continue
+            key = "%s_%s" % (name, kvk) + ("_sparse_top%d" % topk if topk else "")
+            configs[key] = measure_config(mla, name, kvk, topk, dev, stream, peaks)
 
     if rank == 0:
         hbm, tfl_burst, tfl_sust, src = measured_peaks()
@@ -526,28 +669,36 @@ def main():
         else:
             roof = {"bound": "tensor", "achieved": ach_tf, "peak": tfl_burst, "unit": "TFLOP/s",
                     "frac": ach_tf / tfl_burst}
-        roof.update({"traffic": profiled_traffic(args.kv),
-                     "kernel": "mla decode split kernel" + (" (fp8 cache)" if fp8 else ""),
+        roof.update({"traffic": None if topk else profiled_traffic(args.kv),
+                     "kernel": ("mla sparse decode (split + combine kernels, one call)" if topk else
+                                "mla decode split kernel" + (" (fp8 cache)" if fp8 else "")),
                      "peak_source": src + " (MEASURED_PEAKS.json)" if src == "measured" else "fallback",
                      "algorithmic_bytes_per_launch": counts["bytes"], "algorithmic_flops_per_launch": counts["flops"],
                      "launch_ms": split_avg_ms, "hbm_frac": ach_gbs / hbm, "tensor_frac": ach_tf / tfl_burst,
-                     "tensor_frac_sustained": ach_tf / tfl_sust})
-        line = {"metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": "TB/s", "tflops": tflops,
+                     "tensor_frac_sustained": ach_tf / tfl_sust,
+                     "hbm_frac_spec": ach_gbs / SPEC_HBM_GBS, "tensor_frac_spec": ach_tf / SPEC_BF16_TFLOPS,
+                     "spec_peaks": {"hbm_gbs": SPEC_HBM_GBS, "bf16_tflops": SPEC_BF16_TFLOPS}})
+        line = {"metric": METRIC_SPARSE if topk else (METRIC_FP8 if fp8 else METRIC), "value": value, "unit": "TB/s", "tflops": tflops,
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f16 (fp8 E4M3 cache)" if fp8 else "bf16", "data": "synthetic",
-                "config": {"workload": describe(wl, args.kv), "kv": args.kv, "batch": wl.batch, "h_q": wl.h_q, "s_q": wl.s_q,
+                "config": {"workload": describe(wl, args.kv) + (", top-%d sparse lists (uniform, sorted)" % topk
+                                                                 if topk else ""), "kv": args.kv, "topk": topk or None, "batch": wl.batch, "h_q": wl.h_q, "s_q": wl.s_q,
                            "causal": wl.causal, "num_parts": num_parts, "fixed_cost": fixed_cost,
                            "l2": ("inputs larger than L2 (KV cache %.0f MB > 126 MB); no flush" % (counts["kv_bytes"] / 1e6)
                                   if flush is None else "inputs (%.1f MB) fit in L2: a 256 MB write flushes L2 between "
                                   "steps, outside the timed steps" % (in_bytes / 1e6)),
                            "parallelism": "independent batch per GPU" if world > 1 else "1 GPU"},
                 "roofline": roof, "clocks": clk.summary(), "e2e": e2e, "gpu_launches": launches,
+                "target": {"what": "split kernel >= %.2f of the measured HBM peak on v3" % TARGET_HBM_FRAC,
+                           "hbm_frac": ach_gbs / hbm,
+                           "met": bool(args.workload == "v3" and ach_gbs / hbm >= TARGET_HBM_FRAC)},
+                "configs": configs,
                 "neighbours": neighbours,
                 "graph": None if graph_ms is None else {
                     "ms_per_step": graph_ms, "value": job_throughput(counts["bytes"], world, graph_ms), "unit": "TB/s",
                     "note": "the same step (metadata + split + combine) captured once in a CUDA graph and replayed"}}
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not topk:
             line["cpu_baseline"] = cpu_baseline(wl, inp, kv=args.kv)
         print(json.dumps(line), flush=True)
     if dist is not None:
