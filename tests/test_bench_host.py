@@ -12,7 +12,19 @@ def test_code_only_ignores_comments_and_whitespace_but_not_code():
 
 
 def test_source_hash_covers_the_split_kernel_files():
-    assert set(bench.SPLIT_KERNEL_SOURCES) == {"common.cuh", "decode_sm100.cu", "sm100_ptx.cuh"}
+    """The hash covers decode_sm100.cu and every local header it includes, transitively."""
+    import os
+    import re
+    csrc = os.path.join(os.path.dirname(bench.__file__), "mla_decode_attention_14_b200", "csrc")
+    need, todo = set(), ["decode_sm100.cu"]
+    while todo:
+        name = todo.pop()
+        if name in need:
+            continue
+        need.add(name)
+        with open(os.path.join(csrc, name)) as f:
+            todo += [m for m in re.findall(r'#include "([^"/]+)"', f.read())]
+    assert need <= set(bench.SPLIT_KERNEL_SOURCES), sorted(need - set(bench.SPLIT_KERNEL_SOURCES))
     h = bench.kernel_source_hash()
     assert len(h) == 16 and h == bench.kernel_source_hash()
 
