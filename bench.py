@@ -650,11 +650,11 @@ def main():
     if world == 1 and not args.no_configs and not topk:
         peaks = measured_peaks()
         configs = {}
-        for name, kvk, topk in CONFIG_SET:
-            if name == args.workload and kvk == args.kv and topk is None:
+        for name, kvk, ck in CONFIG_SET:
+            if name == args.workload and kvk == args.kv and ck is None:
                 continue
-            key = "%s_%s" % (name, kvk) + ("_sparse_top%d" % topk if topk else "")
-            configs[key] = measure_config(mla, name, kvk, topk, dev, stream, peaks)
+            key = "%s_%s" % (name, kvk) + ("_sparse_top%d" % ck if ck else "")
+            configs[key] = measure_config(mla, name, kvk, ck, dev, stream, peaks)
 
     if rank == 0:
         hbm, tfl_burst, tfl_sust, src = measured_peaks()
