@@ -210,6 +210,7 @@ DecodeParams make_params(const void *q, const void *kv, int64_t num_blocks, cons
     p.v_scale = 1.f;
     p.q_lat_mul = 1.f;
     p.q_rope_mul = 1.f;
+    p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31) == 0;
     p.indices = nullptr;  // dense
     p.topk = 0;
     p.sp_sq = 0;

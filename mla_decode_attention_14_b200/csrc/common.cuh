@@ -44,6 +44,7 @@ struct DecodeParams {
     int64_t bt_stride;
     int batch, s_q, h_q, rows, num_parts;
     int causal;
+    int out_v8;                    // `out` is 32-byte aligned: the epilogue may use 32-byte stores
     float scale;                   // softmax scale
     float scale_log2;              // scale * log2(e) (fp8 cache: also times 2^-k, see q_rope_mul)
     // fp8 cache only: a latent byte x stands for kv_scale * e4m3(x), kv_scale = q_lat_mul * 2^-k with

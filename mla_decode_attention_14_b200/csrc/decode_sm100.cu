@@ -303,12 +303,15 @@ __device__ void gather_producer(Smem &sm, const DecodeParams &p, const int32_t *
 __device__ void zero_tail_rows(uint8_t *st, int valid, int lane) {
     const int zr = kBlk - valid;
     const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int e = lane; e < 4 * zr * 8; e += 32) {  // four 128-byte-swizzled boxes: 8 chunks per row
-        const int b = e / (zr * 8), rem = e % (zr * 8);
-        *reinterpret_cast<uint4 *>(st + b * kBoxBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
+    // (whole rows are zeroed, so the swizzle, a permutation within each row, does not matter; shifts,
+    // not divisions: this runs on Gemm2's issuing warp right before the last block's MMAs)
+    for (int e = lane; e < zr * 8; e += 32) {  // chunk e % 8 of tail row e / 8 in each of the four boxes
+        const int off = (valid + (e >> 3)) * 128 + ((e & 7) << 4);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) *reinterpret_cast<uint4 *>(st + b * kBoxBytes + off) = z;
     }
     for (int e = lane; e < zr * 4; e += 32)  // rotary box: 4 chunks per 64-byte row
-        *reinterpret_cast<uint4 *>(st + 4 * kBoxBytes + (valid + e / 4) * 64 + (e % 4) * 16) = z;
+        *reinterpret_cast<uint4 *>(st + 4 * kBoxBytes + (valid + (e >> 2)) * 64 + ((e & 3) << 4)) = z;
     fence_proxy_async_smem();  // generic-proxy writes visible to the tensor core
     __syncwarp();
 }
@@ -533,6 +536,17 @@ __device__ __forceinline__ void load_q(Smem &sm, const SoftCtx &c, const Piece &
     if (c.lane == 0) mbar_arrive(&sm.q_full);
 }
 
+// Brings this thread's part of piece `pc`'s query row into L2 ahead of load_q (its 256 bytes of latent
+// dims and 32 bytes of rotary dims): load_q's four dependent rounds of loads then hit L2.
+__device__ __forceinline__ void prefetch_q(const SoftCtx &c, const Piece &pc) {
+    if (!c.row_ok) return;
+    const DecodeParams &p = *c.p;
+    const char *row = reinterpret_cast<const char *>(p.q + ((size_t)pc.seq * p.rows + c.r) * kDqk);
+    prefetch_l2(row + 2 * (256 * (int)c.half + 128 * c.th));
+    prefetch_l2(row + 2 * (256 * (int)c.half + 128 * c.th) + 128);
+    prefetch_l2(row + 2 * (512 + 32 * (int)c.half + 16 * c.th));
+}
+
 // Own partial scores of block g for this thread's 32 tokens (raw, unscaled); keys at or past `vis`
 // become -inf. The accumulators are released as soon as the scores are in registers.
 // Sparse mode: keys are the stage's validity mask bits instead (then `nvalid` holds this thread's
@@ -681,6 +695,11 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
     w.init(meta, p);
     if (!w.live) return;
     load_q<F8>(sm, c, w.pc);
+    if constexpr (!F8) {  // (measured: the fp8 kernel ran 12% slower with these prefetches in its loop)
+        Cursor<SP> tmp = w.cur;
+        Piece nx;
+        if (tmp.next(p, nx)) prefetch_q(c, nx);
+    }
     int vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
     float e_own[kTokPer], m_own;
     int nv_own;  // valid tokens of the block being finished, among this thread's 32
@@ -704,7 +723,14 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
         float snx[kTokPer];
         int nv_nx = 0;
         if (nx_live) {
-            if (w.first()) vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
+            if (w.first()) {  // block g+1 starts a piece: its query was loaded; warm the next piece's
+                vis = c.row_ok ? visible_keys(w.pc.n, p.s_q, t_q, p.causal) : 0;
+                if constexpr (!F8) {
+                    Cursor<SP> tmp = w.cur;
+                    Piece nx;
+                    if (tmp.next(p, nx)) prefetch_q(c, nx);
+                }
+            }
             if (!load_raw<SP>(sm, c, g + 1, w.blk * kBlk, vis, snx, nv_nx)) return;
             if (w.last()) {
                 Cursor<SP> tmp = w.cur;
@@ -944,29 +970,29 @@ __device__ void softmax_role(Smem &sm, const DecodeParams &p, const int32_t *met
                     tmem_ld16(tmem + kTmemO + c.lane_off + col, v);
                     tmem_wait_ld();
                     if (!c.row_ok) continue;
+                    // 32-byte stores: each lane writes its own row, so a warp's store touches 32 rows and
+                    // the number of stores, not their width, sets the epilogue's time
                     if (whole) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)a_seq * p.rows + c.r) * kDv +
-                                                               256 * half + col);
+                        uint32_t wv[8];
 #pragma unroll
-                        for (int q4 = 0; q4 < 2; ++q4) {
-                            uint32_t wv[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                __nv_bfloat162 two =
-                                    __floats2bfloat162_rn(__uint_as_float(v[8 * q4 + 2 * j]) * inv,
-                                                          __uint_as_float(v[8 * q4 + 2 * j + 1]) * inv);
-                                wv[j] = *reinterpret_cast<uint32_t *>(&two);
-                            }
-                            dst[q4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        for (int j = 0; j < 8; ++j) {
+                            __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * inv,
+                                                                       __uint_as_float(v[2 * j + 1]) * inv);
+                            wv[j] = *reinterpret_cast<uint32_t *>(&two);
+                        }
+                        __nv_bfloat16 *dst = p.out + ((size_t)a_seq * p.rows + c.r) * kDv + 256 * half + col;
+                        if (p.out_v8) {
+                            st_global_v8(dst, wv);
+                        } else {  // `out` only 16-byte aligned
+                            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
                         }
                     } else {
-                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((size_t)a_slot * p.rows + c.r) * kDv +
-                                                                 256 * half + col);
+                        float *dst = p.o_part + ((size_t)a_slot * p.rows + c.r) * kDv + 256 * half + col;
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            dst[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
-                                                  __uint_as_float(v[4 * q4 + 2]) * inv,
-                                                  __uint_as_float(v[4 * q4 + 3]) * inv);
+                        for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * inv);
+                        st_global_v8(dst, v);
+                        st_global_v8(dst + 8, v + 8);
                     }
                 }
                 if (c.row_ok && half == 0 && c.th == 0) {

@@ -154,3 +154,22 @@ def test_bounded_wait_times_out_and_the_context_survives():
     assert mla.check_status() == 0  # read and cleared
     wl = W.workload("tiny")
     parity.full_parity(W.make_inputs(wl, seed=2, tail="nan"), what="after a timeout")
+
+
+def test_output_only_16_byte_aligned():
+    """`out` 16-byte but not 32-byte aligned (allowed by the ABI): the epilogue falls back from
+    32-byte to 16-byte stores and the result is unchanged."""
+    wl = W.custom(3, 128, 1, [300, 64, 5])
+    inp = W.make_inputs(wl, seed=13, tail="nan")
+    q, kv, bt, sl = parity.to_device(inp)
+    meta = mla.get_metadata(sl, 128, 1)
+    n = 3 * 128 * 512
+    buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    out = buf[8:].view(3, 1, 128, 512)
+    assert out.data_ptr() % 32 == 16
+    _, lse = mla.decode(q, kv, bt, sl, inp["scale"], False, meta, out=out)
+    assert mla.check_status() == 0
+    ref_o, ref_l = oracle.decode(inp["q"], inp["kv"], inp["block_table"], inp["seqlens"], inp["scale"], False)
+    parity.compare(parity.bf16_to_f64(out), lse.cpu().numpy().astype(np.float64), ref_o, ref_l, "16-byte aligned out")
+    aligned_out, _ = mla.decode(q, kv, bt, sl, inp["scale"], False, meta)
+    assert torch.equal(aligned_out, out)
