@@ -248,14 +248,16 @@ int mla_default_num_parts(int device, int h_q, int s_q, int *num_parts) {
     return MLA_OK;
 }
 
-// Measured on a B200 (whole step: metadata + split + combine), the best start-up cost was 12
-// blocks for 128 query rows (U[1024, 8192] lengths), 8 for 64 rows with lognormal lengths and
-// 3-20 made no difference for 16 rows: a piece's start (Q load, pipeline fill, partial writes,
-// one more combine input) costs about as much as ten blocks of steady-state work.
+// Measured on a B200 (whole step: metadata + split + combine) once a piece's start had been made
+// cheap (the next piece's query prefetched into L2, 32-byte epilogue stores, tail zeroing without
+// divisions): start-up costs of 3 / 5 / 10 blocks gave 0.273 / 0.277 / 0.303 ms for 128 query rows
+// (U[1024, 8192] lengths), 0.152 / 0.141 / 0.148 ms for 64 rows with lognormal lengths and
+// 0.119 / 0.121 / 0.126 ms for 16 rows: a piece's start (Q load, pipeline fill, partial writes, one
+// more combine input) now costs about as much as five blocks of steady-state work.
 int mla_default_fixed_cost(int h_q, int s_q) {
     (void)h_q;
     (void)s_q;
-    return 10;
+    return 5;
 }
 
 size_t mla_workspace_bytes(int batch, int s_q, int h_q, int num_parts) {
