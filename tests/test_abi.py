@@ -144,3 +144,35 @@ def test_head_gemm_arguments_checked_on_host(L):
     for bad in (dict(x=None), dict(w=None), dict(y=None), dict(m=0), dict(heads=0), dict(k=96), dict(n=100),
                 dict(ldx=2044), dict(xh=100), dict(ldx=1024), dict(ldy=4096), dict(x=FAKE + 8)):
         assert call(**bad) == 1, bad  # MLA_ERR_INVALID_ARG
+
+
+def _sparse_call(L, **kw):
+    a = dict(q=FAKE, kv=FAKE, nblk=10, bt=FAKE, bts=4, sl=FAKE, ix=FAKE, topk=64, tm=FAKE, ns=FAKE, P=4, b=2,
+             s_q=2, h_q=16, scale=0.1, out=FAKE, lse=FAKE, ws=FAKE, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return L.mla_decode_sparse(a["q"], a["kv"], a["nblk"], a["bt"], a["bts"], a["sl"], a["ix"], a["topk"], a["tm"],
+                               a["ns"], a["P"], a["b"], a["s_q"], a["h_q"], a["scale"], a["out"], a["lse"], a["ws"],
+                               a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(ix=None), dict(ix=FAKE + 2), dict(topk=0), dict(topk=(1 << 24) + 1), dict(q=None), dict(kv=FAKE + 2),
+    dict(b=0), dict(s_q=0), dict(h_q=0), dict(h_q=1025), dict(b=1 << 20, s_q=1 << 10), dict(P=0), dict(nblk=0),
+    dict(scale=float("nan")), dict(out=FAKE + 8),
+])
+def test_sparse_invalid_arguments_rejected_on_host(L, bad):
+    assert _sparse_call(L, **bad) == 1  # MLA_ERR_INVALID_ARG
+
+
+def test_sparse_workspace_is_that_of_its_work_units(L):
+    # batch * s_q work units of h_q rows: the dense formula at (batch * s_q, 1, h_q)
+    need = L.mla_workspace_bytes(2 * 2, 1, 16, 4)
+    assert _sparse_call(L, wsb=need - 256) == 3  # MLA_ERR_WORKSPACE
+
+
+def test_sparse_metadata_argument_checks(L):
+    assert L.mla_get_metadata_sparse(2, 1, 16, 64, 4, 5, None, FAKE, None) == 1
+    assert L.mla_get_metadata_sparse(2, 1, 16, 0, 4, 5, FAKE, FAKE, None) == 1
+    assert L.mla_get_metadata_sparse(0, 1, 16, 64, 4, 5, FAKE, FAKE, None) == 1
+    assert L.mla_get_metadata_sparse(2, 1, 16, 64, 0, 5, FAKE, FAKE, None) == 1
+    assert L.mla_get_metadata_sparse(2, 1, 16, 64, 4, -1, FAKE, FAKE, None) == 1
