@@ -35,6 +35,7 @@ struct Params {
     int64_t ldy, y_head;  // elements
     int64_t x_head;       // elements: column of head h's X_h within a row of X
     int m, n, k, heads;
+    int y_v8;             // y, ldy and y_head allow 32-byte stores (else 16-byte ones)
 };
 
 __global__ void __launch_bounds__(128, 1)
@@ -118,9 +119,14 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constan
                     __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
                     w[j] = *reinterpret_cast<uint32_t *>(&two);
                 }
-                uint4 *dst = reinterpret_cast<uint4 *>(p.y + (int64_t)r * p.ldy + h * p.y_head + n0 + 16 * c16);
-                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                // each lane writes its own row, so the number of stores sets the epilogue's time
+                __nv_bfloat16 *dst = p.y + (int64_t)r * p.ldy + h * p.y_head + n0 + 16 * c16;
+                if (p.y_v8) {
+                    st_global_v8(dst, w);
+                } else {
+                    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                }
             }
         }
     }
@@ -148,6 +154,7 @@ cudaError_t launch_head_gemm(const CUtensorMap &map_x, const CUtensorMap &map_w,
     p.n = n;
     p.k = k;
     p.heads = heads;
+    p.y_v8 = (reinterpret_cast<uintptr_t>(y) % 32) == 0 && (ldy * 2) % 32 == 0 && (y_head * 2) % 32 == 0;
     const size_t smem = head_gemm_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(hg::head_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
