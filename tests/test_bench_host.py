@@ -32,3 +32,27 @@ def test_source_hash_covers_the_split_kernel_files():
 def test_job_throughput_counts_every_rank():
     # 1 GB per rank, 4 ranks, 2 ms per step -> 2 TB/s
     assert abs(bench.job_throughput(10 ** 9, 4, 2.0) - 2.0) < 1e-12
+
+
+def test_roofline_fractions_against_both_peaks():
+    peaks = (6535.7, 1638.2, 1368.0, "measured")
+    # 1 GB and 1 TFLOP in 1 ms: 1000 GB/s and 1000 TFLOP/s
+    r = bench.roofline_fracs(10 ** 9, 10 ** 12, 1e-3, peaks)
+    assert abs(r["hbm_frac"] - 1000 / 6535.7) < 1e-12
+    assert abs(r["tensor_frac"] - 1000 / 1638.2) < 1e-12
+    assert abs(r["hbm_frac_spec"] - 1000 / bench.SPEC_HBM_GBS) < 1e-12
+    assert abs(r["tensor_frac_spec"] - 1000 / bench.SPEC_BF16_TFLOPS) < 1e-12
+    assert r["bound"] == "tensor"  # 1000 flop/B is above the ridge (~251)
+    assert bench.roofline_fracs(10 ** 9, 10 ** 10, 1e-3, peaks)["bound"] == "hbm"
+
+
+def test_config_set_names_known_workloads():
+    from mla_decode_attention_14_b200 import workloads as W
+    keys = set()
+    for name, kv, topk in bench.CONFIG_SET:
+        assert name in W.NAMES and kv in ("bf16", "fp8")
+        assert topk is None or (kv == "bf16" and topk > 0)
+        keys.add((name, kv, topk))
+    assert len(keys) == len(bench.CONFIG_SET)
+    # every workload appears in both cache formats, apart from tiny (bf16 only)
+    assert {n for n, k, t in bench.CONFIG_SET if k == "fp8"} == set(W.NAMES) - {"tiny"}
