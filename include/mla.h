@@ -31,10 +31,12 @@
  *      accumulators (same section, feature (4)), an fp32 online softmax; pieces of
  *      split sequences leave fp32 partial outputs + lse in the workspace, and a
  *      combine kernel merges them by log-sum-exp.
- * Around it: mla_decode_fp8 reads an FP8 (E4M3) latent cache instead; mla_append_kv /
- * mla_append_kv_fp8 write new tokens into the cache; mla_head_gemm computes the per-head
- * projections on either side (the absorbed q_nope W_UK and o_latent W_UV); mla_decode_host
- * and mla_decode_noalloc are conveniences over mla_decode.
+ * Around it: mla_decode_fp8 reads an FP8 (E4M3) latent cache instead; mla_decode_sparse
+ * attends each query token to a list of cache positions (top-k) instead of its whole
+ * sequence; mla_append_kv / mla_append_kv_fp8 write new tokens into the cache;
+ * mla_head_gemm computes the per-head projections on either side (the absorbed q_nope W_UK
+ * and o_latent W_UV); mla_decode_host and mla_decode_noalloc are conveniences over
+ * mla_decode.
  *
  * Conventions for every call:
  *   - Pointers are DEVICE pointers unless the name says host. All device buffers are
